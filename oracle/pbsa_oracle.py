@@ -1,0 +1,483 @@
+"""CPU oracle for Persistent Block-Sparse Attention (PBSA) -- TEST INFRASTRUCTURE.
+
+Only the tests, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this module.  The product path (the CUDA library and
+its Python binding) never calls it, and this module imports nothing of the
+product.
+
+What it computes is the hot path of Sparse Forcing's PBSA, restated step by
+step in plain float64 numpy with Python loops over (batch, head, block):
+
+* a1/a2  block compression by pooling and coarse block scoring
+         (Sparse Forcing, gist.science/es, section 2 "Persistente Block-Sparse
+         Attention (PBSA)", item "Compresión de Bloques"; the abstract on the
+         shd-paper.top page: pooled routing is the PBSA kernel's job);
+* a3     the persistent memory P_t: sink blocks, dynamic blocks chosen by
+         coarse scoring, Top-C retention, and the learned compression,
+         retention and refresh of the persistent blocks (same page, section 2 "Arquitectura
+         Propuesta", items "Memoria Persistente", "Bloques Sumidero",
+         "Bloques Dinámicos", "Mecanismo de Actualización"; the abstract);
+* a4/a5  the local window L_t with a per-query-block Top-K of relevant blocks
+         (section 2 "Arquitectura Propuesta", item "Ventana Local");
+* a6     hybrid attention: dense over the persistent memory, sparse over the
+         local window (section 2 PBSA, item "Atención Híbrida");
+* a7     the backward pass of a6 for the trainable path (section 3
+         "Contribuciones Clave", item "Kernel PBSA"; section 2 "Entrenamiento").
+
+The pages give no formulas.  Where they are silent this module takes the
+plainest reading; each reading is named in the docstring of the function that
+takes it (R1..R19 are the names used in the design notes).
+
+Every function here is pinned by the tests under ``tests/test_oracle_*.py``
+against closed forms, invariants, brute force and library routines (torch's
+scaled-dot-product attention and autograd in float64); none is left unpinned.
+"""
+from __future__ import annotations
+
+import math
+from typing import Optional, Tuple
+
+import numpy as np
+
+EVICT = 0
+MERGE_MEAN = 1
+MASK_CHUNK = 0
+MASK_TOKEN = 1
+
+
+# ---------------------------------------------------------------------------
+# storage rounding
+# ---------------------------------------------------------------------------
+
+def round_bf16(x: np.ndarray) -> np.ndarray:
+    """Round float64 values to the nearest bfloat16 (ties to even), returned as float64.
+
+    A bfloat16 keeps 8 significant bits.  ``frexp`` writes x = m * 2**e with
+    0.5 <= |m| < 1, so m * 256 holds exactly the 8 kept bits left of the
+    point; ``np.round`` rounds half to even."""
+    x = np.asarray(x, dtype=np.float64)
+    m, e = np.frexp(x)
+    return np.ldexp(np.round(m * 256.0) / 256.0, e)
+
+
+def round_storage(x: np.ndarray, dtype: str) -> np.ndarray:
+    if dtype == "bf16":
+        return round_bf16(x)
+    if dtype == "f32":
+        return np.asarray(x, dtype=np.float32).astype(np.float64)
+    if dtype == "f64":
+        return np.asarray(x, dtype=np.float64)
+    raise ValueError(dtype)
+
+
+# ---------------------------------------------------------------------------
+# a1  block compression by pooling
+# ---------------------------------------------------------------------------
+
+def query_block_lengths(Tq: int, bs: int) -> np.ndarray:
+    """Query rows are tiled into ceil(Tq/bs) blocks, the last one partial (R9)."""
+    n = -(-Tq // bs)
+    lens = np.full(n, bs, dtype=np.int64)
+    if n:
+        lens[-1] = Tq - (n - 1) * bs
+    return lens
+
+
+def pool_queries(q: np.ndarray, bs: int) -> np.ndarray:
+    """Mean of the query rows of each query block (R1: mean over valid tokens).
+
+    q: [B,H,Tq,D] -> q_bar [B,H,nQB,D] float64."""
+    B, H, Tq, D = q.shape
+    lens = query_block_lengths(Tq, bs)
+    out = np.zeros((B, H, len(lens), D))
+    for b in range(B):
+        for h in range(H):
+            for i, n in enumerate(lens):
+                rows = q[b, h, i * bs:i * bs + n].astype(np.float64)
+                out[b, h, i] = rows.sum(axis=0) / n
+    return out
+
+
+def pool_keys(kpool: np.ndarray, blk_len: np.ndarray, ids, k_bar: np.ndarray) -> np.ndarray:
+    """Mean of the valid key rows of each listed block; other entries of k_bar are kept.
+
+    kpool: [B,H,NB,bs,D]; blk_len: [B,H,NB]; k_bar: [B,H,NB,D] (copied).
+    A block of length 0 pools to the zero vector."""
+    out = np.array(k_bar, dtype=np.float64, copy=True)
+    B, H = kpool.shape[:2]
+    for b in range(B):
+        for h in range(H):
+            for j in ids:
+                n = int(blk_len[b, h, j])
+                if n == 0:
+                    out[b, h, j] = 0.0
+                else:
+                    out[b, h, j] = kpool[b, h, j, :n].astype(np.float64).sum(axis=0) / n
+    return out
+
+
+# ---------------------------------------------------------------------------
+# a2  coarse block scores and the memory score
+# ---------------------------------------------------------------------------
+
+def block_scores(q_bar: np.ndarray, k_bar: np.ndarray, scale: float) -> np.ndarray:
+    """S[b,h,i,j] = scale * <q_bar_i, k_bar_j> for every pair (R2)."""
+    B, H, nQB, D = q_bar.shape
+    NB = k_bar.shape[2]
+    S = np.zeros((B, H, nQB, NB))
+    for b in range(B):
+        for h in range(H):
+            S[b, h] = scale * (q_bar[b, h] @ k_bar[b, h].T)
+    return S
+
+
+def memory_scores(S: np.ndarray) -> np.ndarray:
+    """Relevance of a block to the current step: mean of its scores over the
+    query blocks of the chunk (R3).  S: [B,H,nQB,NB] -> m [B,H,NB]."""
+    return S.sum(axis=2) / S.shape[2]
+
+
+def score_blocks(q, kpool, blk_len, pool_ids, k_bar, scale, bs):
+    """The whole scoring call: pool Q, (re)pool the listed key blocks, score all blocks."""
+    q_bar = pool_queries(q, bs)
+    k_bar = pool_keys(kpool, blk_len, pool_ids, k_bar)
+    S = block_scores(q_bar, k_bar, scale)
+    return q_bar, k_bar, S, memory_scores(S)
+
+
+# ---------------------------------------------------------------------------
+# a3  persistent-memory update
+# ---------------------------------------------------------------------------
+
+class _Item:
+    """A candidate of the Top-C retention: an occupied slot or a block leaving the window."""
+
+    def __init__(self, phys, src, w, m, old_slot):
+        self.phys = int(phys)        # where its content lives now
+        self.src = int(src)          # global id of the block it came from
+        self.w = float(w)            # number of blocks merged into it
+        self.m = float(m)            # memory score
+        self.old_slot = old_slot     # slot index if it already is in memory
+
+
+def _masked_rows(x: np.ndarray, n: int) -> np.ndarray:
+    y = np.zeros_like(x, dtype=np.float64)
+    y[:n] = x[:n]
+    return y
+
+
+def update_memory(kpool, vpool, blk_len, blk_pos, k_bar, slot_src, slot_w,
+                  cand_ids, cand_src, mem_score, P: int, n_sink: int, policy: int,
+                  store: str):
+    """Top-C retention of the persistent memory P_t, in place on copies of the inputs.
+
+    Sparse Forcing keeps a bounded set of historical blocks: fixed sink
+    anchors plus dynamic blocks chosen by coarse scoring, refreshed by keeping
+    the C best-scoring blocks and discarding the rest as they leave the local
+    window (gist.science/es, section 2 "Arquitectura Propuesta"); per the
+    abstract the mechanism also compresses persistent blocks, not only keeps them.
+
+    Readings taken:
+      R4  C = P - n_sink dynamic blocks besides the sinks.
+      R6  slot s < n_sink is the sink of global block s: that block enters its
+          sink slot when it leaves the window and is never ranked or merged into.
+      R3  candidates are ranked by the memory score m (mean block score over the
+          query blocks of the step); key (m descending, source id ascending).
+      --  kept blocks already in memory stay in their slot; newly kept blocks
+          fill the free non-sink slots in ascending slot order, taken in
+          ascending source-id order.
+      R5  policy MERGE_MEAN: each loser j is merged into the kept slot whose
+          pre-merge pooled key has the largest dot product with j's pooled key
+          (ties: lowest slot).  A slot's new content is the weight-averaged
+          token-position-wise mean of its blocks, rows past a block's length
+          counting as zero; weights add, the length is the maximum, the pooled
+          key is recomputed from the stored result.  Policy EVICT drops losers.
+
+    Shapes: kpool/vpool [B,H,NB,bs,D]; blk_len/blk_pos [B,H,NB]; k_bar
+    [B,H,NB,D]; slot_src/slot_w [B,H,P]; cand_ids/cand_src [n]; mem_score
+    [B,H,NB].  ``store`` is the storage type new slot rows are rounded to.
+
+    Returns (kpool, vpool, blk_len, blk_pos, k_bar, slot_src, slot_w, info) with
+    ``info[(b,h)] = dict(kept=[src...], losers=[src...], target={src: slot})``.
+    """
+    kp = np.array(kpool, dtype=np.float64, copy=True)
+    vp = np.array(vpool, dtype=np.float64, copy=True)
+    ln = np.array(blk_len, copy=True)
+    ps = np.array(blk_pos, copy=True)
+    kb = np.array(k_bar, dtype=np.float64, copy=True)
+    ss = np.array(slot_src, copy=True)
+    sw = np.array(slot_w, dtype=np.float64, copy=True)
+    B, H = kp.shape[:2]
+    info = {}
+    for b in range(B):
+        for h in range(H):
+            items = []
+            sinks_in = []
+            for s in range(n_sink, P):
+                if ss[b, h, s] >= 0:
+                    items.append(_Item(s, ss[b, h, s], sw[b, h, s], mem_score[b, h, s], s))
+            for c, src in zip(cand_ids, cand_src):
+                if src < n_sink:
+                    sinks_in.append((int(src), int(c)))
+                else:
+                    items.append(_Item(c, src, 1.0, mem_score[b, h, c], None))
+            order = sorted(items, key=lambda it: (-it.m, it.src))
+            n_keep = min(P - n_sink, len(order))
+            kept, losers = order[:n_keep], order[n_keep:]
+
+            slot_of = {}
+            taken = {it.old_slot for it in kept if it.old_slot is not None}
+            free = [s for s in range(n_sink, P) if s not in taken]
+            for it in kept:
+                if it.old_slot is not None:
+                    slot_of[id(it)] = it.old_slot
+            for it, s in zip(sorted([it for it in kept if it.old_slot is None],
+                                    key=lambda it: it.src), free):
+                slot_of[id(it)] = s
+
+            merged_into = {s: [] for s in range(P)}
+            target = {}
+            if policy == MERGE_MEAN and kept:
+                by_slot = sorted(kept, key=lambda it: slot_of[id(it)])
+                for j in losers:
+                    best, best_dot = None, -math.inf
+                    for c in by_slot:
+                        d = float(np.dot(kb[b, h, j.phys], kb[b, h, c.phys]))
+                        if d > best_dot:
+                            best, best_dot = c, d
+                    s = slot_of[id(best)]
+                    merged_into[s].append(j)
+                    target[j.src] = s
+
+            # read every source before any slot is written
+            K = {id(it): kp[b, h, it.phys].copy() for it in items}
+            V = {id(it): vp[b, h, it.phys].copy() for it in items}
+            L = {id(it): int(ln[b, h, it.phys]) for it in items}
+            POS = {id(it): int(ps[b, h, it.phys]) for it in items}
+            KB = {id(it): kb[b, h, it.phys].copy() for it in items}
+            sink_K = {s: (kp[b, h, c].copy(), vp[b, h, c].copy(), int(ln[b, h, c]),
+                          int(ps[b, h, c]), kb[b, h, c].copy()) for s, c in sinks_in}
+
+            holder = {slot_of[id(it)]: it for it in kept}
+            for s in range(n_sink, P):
+                if s not in holder:
+                    ss[b, h, s] = -1
+                    sw[b, h, s] = 0.0
+                    ln[b, h, s] = 0
+                    ps[b, h, s] = 0
+                    kb[b, h, s] = 0.0
+                    continue
+                c = holder[s]
+                group = merged_into[s]
+                if not group:
+                    kp[b, h, s] = K[id(c)]
+                    vp[b, h, s] = V[id(c)]
+                    ln[b, h, s] = L[id(c)]
+                    kb[b, h, s] = KB[id(c)]
+                    sw[b, h, s] = c.w
+                else:
+                    W = c.w + sum(j.w for j in group)
+                    ksum = c.w * _masked_rows(K[id(c)], L[id(c)])
+                    vsum = c.w * _masked_rows(V[id(c)], L[id(c)])
+                    for j in group:
+                        ksum += j.w * _masked_rows(K[id(j)], L[id(j)])
+                        vsum += j.w * _masked_rows(V[id(j)], L[id(j)])
+                    n = max([L[id(c)]] + [L[id(j)] for j in group])
+                    kp[b, h, s] = round_storage(ksum / W, store)
+                    vp[b, h, s] = round_storage(vsum / W, store)
+                    ln[b, h, s] = n
+                    kb[b, h, s] = kp[b, h, s, :n].sum(axis=0) / n
+                    sw[b, h, s] = W
+                ss[b, h, s] = c.src
+                ps[b, h, s] = POS[id(c)]
+            for s, (k_, v_, l_, p_, kb_) in sink_K.items():
+                kp[b, h, s], vp[b, h, s] = k_, v_
+                ln[b, h, s], ps[b, h, s], kb[b, h, s] = l_, p_, kb_
+                ss[b, h, s] = s
+                sw[b, h, s] = 1.0
+            info[(b, h)] = dict(kept=[it.src for it in kept], losers=[it.src for it in losers],
+                                keys={it.src: it.m for it in items}, target=target,
+                                slot={it.src: slot_of[id(it)] for it in kept})
+    return kp, vp, ln, ps, kb, ss, sw, info
+
+
+# ---------------------------------------------------------------------------
+# a4/a5  local Top-K selection and the attended-block list
+# ---------------------------------------------------------------------------
+
+def select_local(S: np.ndarray, win_ids, k: int, mem_ids: Optional[np.ndarray],
+                 blk_len: np.ndarray, mask: int = MASK_CHUNK, q_pos0: int = 0,
+                 blk_pos: Optional[np.ndarray] = None, bs: int = 0, Tq: int = 0):
+    """Per query block: Top-K window blocks by block score, united with the memory.
+
+    Inside the sliding window only the K most relevant blocks of each query
+    are attended (gist.science/es, section 2 "Arquitectura Propuesta", item
+    "Ventana Local"); attention is dense over the persistent memory (section 2
+    PBSA, item "Atención Híbrida").
+
+    Readings taken:
+      R7   the window list is given by the caller (current chunk included).
+      R8   chunk mask: every window block is allowed.  Token mask: a block is
+           allowed for query block i when its first token is not after the
+           last query token of block i.
+      R10  ranking key (score descending, physical id ascending); blocks of
+           length 0 are never candidates; if K >= #allowed all are taken.
+      R12  the attended list is the union of the memory ids that hold a block
+           (length > 0) and the local selection, ascending, without duplicates.
+
+    S: [B,H,nQB,NB] scores indexed by physical block id; mem_ids: [B,H,n_mem]
+    physical ids (-1 = none) or None.  Returns a list of lists A[b][h][i]."""
+    B, H, nQB, _ = S.shape
+    lens = query_block_lengths(Tq, bs) if mask == MASK_TOKEN else None
+    out = []
+    for b in range(B):
+        ob = []
+        for h in range(H):
+            oh = []
+            mem = []
+            if mem_ids is not None:
+                mem = [int(m) for m in mem_ids[b, h] if m >= 0 and blk_len[b, h, m] > 0]
+            for i in range(nQB):
+                cands = []
+                for j in win_ids:
+                    j = int(j)
+                    if blk_len[b, h, j] <= 0:
+                        continue
+                    if mask == MASK_TOKEN:
+                        last_q = q_pos0 + i * bs + int(lens[i]) - 1
+                        if blk_pos[b, h, j] > last_q:
+                            continue
+                    cands.append(j)
+                order = sorted(cands, key=lambda j: (-S[b, h, i, j], j))
+                local = order[:min(k, len(order))]
+                oh.append(sorted(set(mem) | set(local)))
+            ob.append(oh)
+        out.append(ob)
+    return out
+
+
+def lists_to_arrays(A, Amax: int):
+    """Pack attended lists into idx [B,H,nQB,Amax] (padding -1) and cnt [B,H,nQB]."""
+    B, H, nQB = len(A), len(A[0]), len(A[0][0])
+    idx = np.full((B, H, nQB, Amax), -1, dtype=np.int32)
+    cnt = np.zeros((B, H, nQB), dtype=np.int32)
+    for b in range(B):
+        for h in range(H):
+            for i in range(nQB):
+                a = A[b][h][i]
+                if len(a) > Amax:
+                    raise ValueError("attended list longer than Amax")
+                idx[b, h, i, :len(a)] = a
+                cnt[b, h, i] = len(a)
+    return idx, cnt
+
+
+# ---------------------------------------------------------------------------
+# a6  hybrid (persistent + local) block-sparse attention, forward
+# ---------------------------------------------------------------------------
+
+def _gather_keys(kpool, vpool, blk_len, blk_pos, b, h, ids):
+    ks, vs, pos = [], [], []
+    for j in ids:
+        n = int(blk_len[b, h, j])
+        ks.append(kpool[b, h, j, :n].astype(np.float64))
+        vs.append(vpool[b, h, j, :n].astype(np.float64))
+        p0 = int(blk_pos[b, h, j]) if blk_pos is not None else 0
+        pos.append(p0 + np.arange(n))
+    D = kpool.shape[-1]
+    if not ks:
+        return np.zeros((0, D)), np.zeros((0, D)), np.zeros(0, dtype=np.int64)
+    return np.concatenate(ks), np.concatenate(vs), np.concatenate(pos)
+
+
+def _logits(qi, kc, scale, mask, q_rows_pos, k_pos):
+    s = scale * (qi @ kc.T)
+    if mask == MASK_TOKEN:
+        s = np.where(k_pos[None, :] > q_rows_pos[:, None], -np.inf, s)
+    return s
+
+
+def attention_fwd(q, kpool, vpool, blk_len, blk_pos, idx, cnt, scale: float,
+                  mask: int = MASK_CHUNK, q_pos0: int = 0):
+    """One softmax over the union of the attended blocks of each query block (R12).
+
+    O_r = sum_c softmax_c(scale * <Q_r, K_c>) V_c over the valid tokens c of
+    the blocks idx[b,h,i,:cnt] (token mask: only c with position <= the query
+    position).  LSE_r = log sum_c exp(scale * <Q_r, K_c>) (natural log).
+    A row with no visible key gets O = 0 and LSE = -inf.
+
+    q: [B,H,Tq,D]; kpool/vpool [B,H,NB,bs,D]; idx [B,H,nQB,Amax]; cnt [B,H,nQB]."""
+    B, H, Tq, D = q.shape
+    bs = kpool.shape[3]
+    lens = query_block_lengths(Tq, bs)
+    O = np.zeros((B, H, Tq, D))
+    LSE = np.full((B, H, Tq), -np.inf)
+    for b in range(B):
+        for h in range(H):
+            for i, n in enumerate(lens):
+                r0 = i * bs
+                ids = [int(x) for x in idx[b, h, i, :cnt[b, h, i]]]
+                kc, vc, kpos = _gather_keys(kpool, vpool, blk_len, blk_pos, b, h, ids)
+                if kc.shape[0] == 0:
+                    continue
+                qi = q[b, h, r0:r0 + n].astype(np.float64)
+                s = _logits(qi, kc, scale, mask, q_pos0 + r0 + np.arange(n), kpos)
+                for r in range(n):
+                    row = s[r]
+                    if not np.isfinite(row).any():
+                        continue
+                    mx = row.max()
+                    e = np.exp(row - mx)
+                    z = e.sum()
+                    O[b, h, r0 + r] = (e / z) @ vc
+                    LSE[b, h, r0 + r] = mx + math.log(z)
+    return O, LSE
+
+
+# ---------------------------------------------------------------------------
+# a7  backward
+# ---------------------------------------------------------------------------
+
+def attention_bwd(q, kpool, vpool, blk_len, blk_pos, idx, cnt, dO, scale: float,
+                  mask: int = MASK_CHUNK, q_pos0: int = 0):
+    """Gradients of ``attention_fwd`` w.r.t. Q, the key pool and the value pool.
+
+    The attended lists are constants (R13: no gradient through selection).
+    For each query block with P = softmax(scale * Q K^T) over its gathered
+    keys: dV += P^T dO, dP = dO V^T, dS = P * (dP - rowsum(P * dP)),
+    dQ = scale * dS K, dK += scale * dS^T Q; key/value gradients are added back
+    to the block rows they were gathered from."""
+    B, H, Tq, D = q.shape
+    bs = kpool.shape[3]
+    lens = query_block_lengths(Tq, bs)
+    dq = np.zeros((B, H, Tq, D))
+    dk = np.zeros(kpool.shape)
+    dv = np.zeros(vpool.shape)
+    for b in range(B):
+        for h in range(H):
+            for i, n in enumerate(lens):
+                r0 = i * bs
+                ids = [int(x) for x in idx[b, h, i, :cnt[b, h, i]]]
+                kc, vc, kpos = _gather_keys(kpool, vpool, blk_len, blk_pos, b, h, ids)
+                if kc.shape[0] == 0:
+                    continue
+                qi = q[b, h, r0:r0 + n].astype(np.float64)
+                doi = dO[b, h, r0:r0 + n].astype(np.float64)
+                s = _logits(qi, kc, scale, mask, q_pos0 + r0 + np.arange(n), kpos)
+                Pm = np.zeros_like(s)
+                for r in range(n):
+                    if np.isfinite(s[r]).any():
+                        e = np.exp(s[r] - s[r].max())
+                        Pm[r] = e / e.sum()
+                dvc = Pm.T @ doi
+                dP = doi @ vc.T
+                dS = Pm * (dP - (Pm * dP).sum(axis=1, keepdims=True))
+                dq[b, h, r0:r0 + n] = scale * (dS @ kc)
+                dkc = scale * (dS.T @ qi)
+                off = 0
+                for j in ids:
+                    m = int(blk_len[b, h, j])
+                    dk[b, h, j, :m] += dkc[off:off + m]
+                    dv[b, h, j, :m] += dvc[off:off + m]
+                    off += m
+    return dq, dk, dv
