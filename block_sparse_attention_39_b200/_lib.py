@@ -1,0 +1,67 @@
+"""ctypes loader of the PBSA C-ABI library (``libpbsa.so``, built in-tree).
+
+There is no fallback: if the library is missing this module raises, so a
+caller can never silently run anything but the CUDA kernels.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libpbsa.so")
+
+c_int, c_float, c_void_p, c_size_t, c_int64 = (ctypes.c_int, ctypes.c_float, ctypes.c_void_p,
+                                                ctypes.c_size_t, ctypes.c_int64)
+
+
+class PbsaDims(ctypes.Structure):
+    _fields_ = [("B", c_int), ("H", c_int), ("D", c_int), ("bs", c_int), ("scale", c_float),
+                ("dtype", c_int)]
+
+
+P = ctypes.POINTER(PbsaDims)
+
+# name -> (restype, argtypes); mirrors include/pbsa.h
+SIGNATURES = {
+    "pbsa_score_blocks": (c_int, [P, c_void_p, c_int, c_void_p, c_int, c_void_p, c_void_p, c_int,
+                                  c_void_p, c_void_p, c_void_p, c_void_p, c_void_p]),
+    "pbsa_update_memory_workspace": (c_size_t, [P, c_int, c_int]),
+    "pbsa_update_memory": (c_int, [P, c_void_p, c_void_p, c_int, c_void_p, c_void_p, c_void_p,
+                                   c_int, c_int, c_void_p, c_void_p, c_void_p, c_void_p, c_int,
+                                   c_void_p, c_int, c_void_p, c_size_t, c_void_p]),
+    "pbsa_select_local": (c_int, [P, c_void_p, c_int, c_int, c_void_p, c_int, c_int, c_void_p,
+                                  c_int, c_void_p, c_int, c_int, c_void_p, c_int, c_void_p,
+                                  c_void_p, c_int, c_int, c_int, c_void_p]),
+    "pbsa_attn_fwd": (c_int, [P, c_void_p, c_int, c_int, c_void_p, c_void_p, c_int, c_void_p,
+                              c_void_p, c_void_p, c_void_p, c_int, c_int, c_void_p, c_void_p,
+                              c_void_p]),
+    "pbsa_attn_bwd_workspace": (c_size_t, [P, c_int, c_int, c_int]),
+    "pbsa_attn_bwd": (c_int, [P, c_void_p, c_int, c_int, c_void_p, c_void_p, c_int, c_void_p,
+                              c_void_p, c_void_p, c_void_p, c_int, c_int, c_void_p, c_void_p,
+                              c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_size_t,
+                              c_void_p]),
+    "pbsa_get_status": (c_int, [c_void_p]),
+    "pbsa_last_error": (ctypes.c_char_p, []),
+    "pbsa_version": (ctypes.c_char_p, []),
+    "pbsa_set_debug": (None, [c_int, c_int64]),
+}
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libpbsa.so (once).  Raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                f"{LIB_PATH} is missing: build it with `python -m block_sparse_attention_39_b200.build`"
+                " (there is no CPU fallback)")
+        handle = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(handle, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = handle
+    return _lib

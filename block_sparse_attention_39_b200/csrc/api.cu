@@ -1,0 +1,108 @@
+// Library-wide state: the per-device status word, error messages, version,
+// debug hooks, and tensor-map encoding through the driver entry point.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <mutex>
+#include <string>
+
+#include "common.cuh"
+#include "tmap.h"
+
+namespace pbsa {
+
+// One status word per device.  Kernels write PBSA_ERR_TIMEOUT into it with
+// atomicCAS(0 -> code); pbsa_get_status reads and clears it.
+__device__ int g_device_status = 0;
+
+static thread_local std::string t_last_error;
+static int g_debug_flags = 0;
+static int64_t g_wait_limit_ns = 2000000000LL;
+
+void set_error(const std::string& msg) { t_last_error = msg; }
+int debug_flags() { return g_debug_flags; }
+int64_t wait_limit_ns() { return g_wait_limit_ns; }
+
+int* device_status_ptr() {
+  static int* ptrs[64] = {nullptr};
+  static std::mutex mu;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (ptrs[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_device_status) != cudaSuccess) return nullptr;
+    ptrs[dev] = static_cast<int*>(p);
+  }
+  return ptrs[dev];
+}
+
+// ------------------------------------------------------------- tensor maps
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+int make_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
+                      uint32_t box_rows, uint32_t box_cols) {
+  EncodeTiledFn fn = encode_fn();
+  PBSA_CHECK_ARG(fn != nullptr, PBSA_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  PBSA_CHECK_ARG(r == CUDA_SUCCESS, PBSA_ERR_CUDA,
+                 "cuTensorMapEncodeTiled failed with code " + std::to_string(int(r)));
+  return PBSA_OK;
+}
+
+}  // namespace pbsa
+
+extern "C" {
+
+int pbsa_get_status(void* stream) {
+  int* p = pbsa::device_status_ptr();
+  if (p == nullptr) {
+    pbsa::set_error("cannot resolve the device status word");
+    return PBSA_ERR_CUDA;
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int host = 0;
+  cudaError_t e = cudaMemcpyAsync(&host, p, sizeof(int), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(p, 0, sizeof(int), s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) {
+    pbsa::set_error(std::string("pbsa_get_status: ") + cudaGetErrorString(e));
+    return PBSA_ERR_CUDA;
+  }
+  return host;
+}
+
+const char* pbsa_last_error(void) { return pbsa::t_last_error.c_str(); }
+
+const char* pbsa_version(void) { return "pbsa-b200 0.1.0 (sm_100a)"; }
+
+void pbsa_set_debug(int flags, int64_t wait_limit_ns) {
+  pbsa::g_debug_flags = flags;
+  pbsa::g_wait_limit_ns = wait_limit_ns > 0 ? wait_limit_ns : 2000000000LL;
+}
+
+}  // extern "C"

@@ -1,0 +1,148 @@
+// a4 + a5: local Top-K selection inside the sliding window and assembly of the
+// attended-block list (persistent memory united with the local selection).
+//
+// Sparse Forcing restricts attention inside the recent window to the Top-K
+// blocks most relevant to each query (gist.science/es, section 2
+// "Arquitectura Propuesta", item "Ventana Local") and attends the persistent
+// memory densely (PBSA item "Atención Híbrida").
+//
+// One warp per (b, h, query block): the window's scores become 64-bit keys
+// (orderable score, ~id), a warp-wide bitonic sort over 256 keys held in
+// registers picks the Top-K, and a second bitonic sort merges the selection
+// with the memory ids into an ascending, duplicate-free list.
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+
+namespace pbsa {
+namespace {
+
+constexpr int KPL = 8;                  // keys per lane: 256 per warp
+constexpr int kSelWarps = 4;
+
+__global__ void __launch_bounds__(32 * kSelWarps)
+select_kernel(const float* __restrict__ scores, int nQB, int NB, const int32_t* __restrict__ win_ids,
+              int n_win, int k, const int32_t* __restrict__ mem_ids, int n_mem,
+              const int32_t* __restrict__ blk_len, int mask, int q_pos0,
+              const int32_t* __restrict__ blk_pos, int Tq, int bs, int32_t* __restrict__ idx,
+              int32_t* __restrict__ cnt, int Amax, int qb_offset, int nQB_total, int* status) {
+  const int lane = threadIdx.x & 31;
+  const int i = blockIdx.x * kSelWarps + (threadIdx.x >> 5);
+  if (i >= nQB) return;
+  const long bh = blockIdx.y;
+  const float* srow = scores + (bh * nQB + i) * static_cast<long>(NB);
+  const int last_q = q_pos0 + i * bs + min(bs, Tq - i * bs) - 1;
+
+  // ---- Top-K over the window
+  uint64_t key[KPL];
+  int n_ok = 0;
+#pragma unroll
+  for (int r = 0; r < KPL; ++r) {
+    const int e = lane * KPL + r;
+    key[r] = 0;
+    if (e < n_win) {
+      const int j = win_ids[e];
+      if (j < 0 || j >= NB) {
+        report_status(status, PBSA_ERR_ARG);
+        continue;
+      }
+      bool ok = blk_len[bh * NB + j] > 0;
+      if (ok && mask == PBSA_MASK_TOKEN) ok = blk_pos[bh * NB + j] <= last_q;
+      if (ok) {
+        key[r] = score_key(srow[j], static_cast<uint32_t>(j));
+        ++n_ok;
+      }
+    }
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) n_ok += __shfl_xor_sync(0xffffffffu, n_ok, off);
+  warp_bitonic_sort_desc<KPL>(key);
+  const int take = min(k, n_ok);
+
+  // ---- union with the memory ids, ascending (descending sort of ~id)
+#pragma unroll
+  for (int r = 0; r < KPL; ++r) {
+    const int e = lane * KPL + r;
+    uint64_t nk = 0;
+    if (e < take) {
+      nk = 0xffffffffull - key_id(key[r]);
+    } else if (e - take < n_mem) {
+      const int m = mem_ids[bh * n_mem + (e - take)];
+      if (m >= 0 && m < NB && blk_len[bh * NB + m] > 0) nk = 0xffffffffull - static_cast<uint32_t>(m);
+    }
+    key[r] = nk;
+  }
+  warp_bitonic_sort_desc<KPL>(key);
+
+  // ---- dedupe and write
+  uint64_t prev_last = __shfl_up_sync(0xffffffffu, key[KPL - 1], 1);
+  int keep[KPL];
+  int mine = 0;
+#pragma unroll
+  for (int r = 0; r < KPL; ++r) {
+    const uint64_t prev = (r == 0) ? ((lane == 0) ? ~0ull : prev_last) : key[r - 1];
+    keep[r] = (key[r] != 0 && key[r] != prev) ? 1 : 0;
+    mine += keep[r];
+  }
+  int incl = mine;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += v;
+  }
+  const int total = __shfl_sync(0xffffffffu, incl, 31);
+  int pos = incl - mine;
+  int32_t* out = idx + (bh * nQB_total + qb_offset + i) * static_cast<long>(Amax);
+  if (total > Amax) {
+    if (lane == 0) report_status(status, PBSA_ERR_SHAPE);
+    return;
+  }
+#pragma unroll
+  for (int r = 0; r < KPL; ++r) {
+    if (keep[r]) out[pos++] = static_cast<int32_t>(0xffffffffu - static_cast<uint32_t>(key[r]));
+  }
+  for (int e = total + lane; e < Amax; e += 32) out[e] = -1;
+  if (lane == 0) cnt[bh * nQB_total + qb_offset + i] = total;
+}
+
+}  // namespace
+}  // namespace pbsa
+
+extern "C" int pbsa_select_local(const pbsa_dims* d, const float* scores, int nQB, int NB,
+                                 const int32_t* win_ids, int n_win, int k, const int32_t* mem_ids,
+                                 int n_mem, const int32_t* blk_len, int mask, int q_pos0,
+                                 const int32_t* blk_pos, int Tq, int32_t* idx, int32_t* cnt,
+                                 int Amax, int qb_offset, int nQB_total, void* stream) {
+  using namespace pbsa;
+  int rc = common_dims_check(d);
+  if (rc) return rc;
+  PBSA_CHECK_ARG(scores && blk_len && idx && cnt, PBSA_ERR_ARG, "select_local: NULL buffer");
+  PBSA_CHECK_ARG(n_win >= 0 && n_win <= 32 * KPL, PBSA_ERR_SHAPE,
+                 "select_local: n_win must be in [0, 256]");
+  PBSA_CHECK_ARG(n_win == 0 || win_ids, PBSA_ERR_ARG, "select_local: win_ids is NULL");
+  PBSA_CHECK_ARG(n_mem >= 0 && (n_mem == 0 || mem_ids), PBSA_ERR_ARG,
+                 "select_local: mem_ids is NULL");
+  PBSA_CHECK_ARG(k >= 0 && nQB >= 1 && NB >= 1 && Amax >= 1, PBSA_ERR_SHAPE,
+                 "select_local: need k >= 0, nQB >= 1, NB >= 1, Amax >= 1");
+  const int take_max = k < n_win ? k : n_win;
+  PBSA_CHECK_ARG(n_mem + take_max <= Amax && n_mem + take_max <= 32 * KPL, PBSA_ERR_SHAPE,
+                 "select_local: n_mem + min(k, n_win) must be <= min(Amax, 256)");
+  PBSA_CHECK_ARG(mask == PBSA_MASK_CHUNK || mask == PBSA_MASK_TOKEN, PBSA_ERR_ARG,
+                 "select_local: bad mask");
+  PBSA_CHECK_ARG(mask == PBSA_MASK_CHUNK || blk_pos, PBSA_ERR_ARG,
+                 "select_local: token mask needs blk_pos");
+  PBSA_CHECK_ARG(Tq >= 1 && (Tq + d->bs - 1) / d->bs == nQB, PBSA_ERR_SHAPE,
+                 "select_local: nQB must be ceil(Tq / bs)");
+  PBSA_CHECK_ARG(qb_offset >= 0 && qb_offset + nQB <= nQB_total, PBSA_ERR_SHAPE,
+                 "select_local: qb_offset + nQB must be <= nQB_total");
+  PBSA_CHECK_ARG(static_cast<long>(d->B) * d->H <= 65535, PBSA_ERR_SHAPE,
+                 "select_local: B*H must be <= 65535");
+  int* status = device_status_ptr();
+  PBSA_CHECK_ARG(status != nullptr, PBSA_ERR_CUDA, "select_local: no device status word");
+  dim3 grid((nQB + kSelWarps - 1) / kSelWarps, d->B * d->H);
+  select_kernel<<<grid, 32 * kSelWarps, 0, static_cast<cudaStream_t>(stream)>>>(
+      scores, nQB, NB, win_ids, n_win, k, mem_ids, n_mem, blk_len, mask, q_pos0, blk_pos, Tq,
+      d->bs, idx, cnt, Amax, qb_offset, nQB_total, status);
+  PBSA_CHECK_LAUNCH("select_kernel");
+  return PBSA_OK;
+}

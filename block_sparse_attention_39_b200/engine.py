@@ -1,0 +1,168 @@
+"""Per-layer PBSA state on the device and the chunk step that drives it.
+
+A ``PbsaLayer`` owns the device buffers of one attention layer: the block
+pool (persistent slots + window ring or snapshot chunks), its metadata, the
+pooled keys, scores, attended lists, outputs and workspace.  ``step`` runs the
+hot path of one chunk -- score -> update memory -> select -> attend -- as four
+calls into the C ABI; the host side only decides which physical ids are passed
+(ring bookkeeping) and never touches tensor data.
+"""
+from __future__ import annotations
+
+from typing import Optional
+
+import torch
+
+from . import pbsa as K
+from pbsa_inputs import Workload
+
+
+def _i32(x, device):
+    return torch.as_tensor(x, dtype=torch.int32, device=device).contiguous()
+
+
+class PbsaLayer:
+    def __init__(self, w: Workload, device="cuda", P_override: Optional[int] = None):
+        self.w = w
+        self.dev = torch.device(device)
+        B, H, D, bs = w.B, w.H, w.D, w.bs
+        self.tdtype = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+        self.d = K.dims(B, H, D, bs, w.scale, self.tdtype)
+        self.dbf = K.dims(B, H, D, bs, w.scale, torch.bfloat16)
+        self.P = w.n_slots
+        self.NB = w.NB_phys
+        self.nQB = w.nb_c
+        self.Amax = self.P + w.k if w.slots_in_pool else w.P + w.k
+        NB, P = self.NB, self.P
+        dev = self.dev
+        self.kpool = torch.zeros(B, H, NB, bs, D, dtype=self.tdtype, device=dev)
+        self.vpool = torch.zeros_like(self.kpool)
+        self.blk_len = torch.zeros(B, H, NB, dtype=torch.int32, device=dev)
+        self.blk_pos = torch.zeros(B, H, NB, dtype=torch.int32, device=dev)
+        self.k_bar = torch.zeros(B, H, NB, D, dtype=torch.float32, device=dev)
+        self.slot_src = torch.full((B, H, max(P, 1)), -1, dtype=torch.int32, device=dev)
+        self.slot_w = torch.zeros(B, H, max(P, 1), dtype=torch.float32, device=dev)
+        self.q = torch.zeros(B, H, w.chunk_tokens, D, dtype=self.tdtype, device=dev)
+        self.q_bar = torch.zeros(B, H, self.nQB, D, dtype=torch.float32, device=dev)
+        self.scores = torch.zeros(B, H, self.nQB, NB, dtype=torch.float32, device=dev)
+        self.mem = torch.zeros(B, H, NB, dtype=torch.float32, device=dev)
+        self.idx = torch.full((B, H, self.nQB, self.Amax), -1, dtype=torch.int32, device=dev)
+        self.cnt = torch.zeros(B, H, self.nQB, dtype=torch.int32, device=dev)
+        self.o = torch.zeros(B, H, w.chunk_tokens, D, dtype=torch.bfloat16, device=dev)
+        self.lse = torch.zeros(B, H, w.chunk_tokens, dtype=torch.float32, device=dev)
+        self.mem_ids = _i32(torch.arange(P).expand(B, H, P), dev) if P else None
+        max_cand = w.nb_c * (len(w.snapshot_candidate_chunks()) if not w.rollout else 1)
+        self.max_cand = max(max_cand, 1)
+        ws = K.update_memory_workspace(self.d, max(P, 1), self.max_cand)
+        self.ws = torch.empty(ws, dtype=torch.uint8, device=dev)
+        self._ids = {}
+        if self.tdtype != torch.bfloat16:
+            # attention runs on bf16 copies of an fp32 cache (R17)
+            self.q16 = torch.zeros(B, H, w.chunk_tokens, D, dtype=torch.bfloat16, device=dev)
+            self.k16 = torch.zeros(B, H, NB, bs, D, dtype=torch.bfloat16, device=dev)
+            self.v16 = torch.zeros_like(self.k16)
+
+    # ------------------------------------------------------------ id lists
+    def ids(self, key, values):
+        t = self._ids.get(key)
+        if t is None:
+            t = _i32(list(values), self.dev)
+            self._ids[key] = t
+        return t
+
+    def chunk_ids(self, t):
+        return self.ids(("chunk", t % self.w.ring_chunks if self.w.rollout else t),
+                        self.w.chunk_phys_ids(t))
+
+    def window_ids(self, t):
+        chunks = self.w.window_chunks(t)
+        key = ("win",) + tuple(c % self.w.ring_chunks if self.w.rollout else c for c in chunks)
+        return self.ids(key, [p for c in chunks for p in self.w.chunk_phys_ids(c)])
+
+    # ------------------------------------------------------------ state
+    def reset_memory(self):
+        """Empty persistent memory (snapshot steps start from it)."""
+        if self.P:
+            self.slot_src.fill_(-1)
+            self.slot_w.zero_()
+            self.blk_len[:, :, :self.P] = 0
+            self.blk_pos[:, :, :self.P] = 0
+            self.k_bar[:, :, :self.P] = 0
+
+    def set_chunk_meta(self, t):
+        """Lengths and positions of chunk t's blocks (where the ring puts them)."""
+        lens = self.w.chunk_block_lens()
+        for j, pid in enumerate(self.w.chunk_phys_ids(t)):
+            self.blk_len[:, :, pid] = lens[j]
+            self.blk_pos[:, :, pid] = t * self.w.chunk_tokens + j * self.w.bs
+
+    def write_chunk(self, t, k_chunk, v_chunk):
+        """Place a chunk's K/V [B,H,T_c,D] into its blocks (the caller's cache append)."""
+        w = self.w
+        ids = w.chunk_phys_ids(t)
+        lens = w.chunk_block_lens()
+        for j, pid in enumerate(ids):
+            r0 = j * w.bs
+            self.kpool[:, :, pid, :lens[j]] = k_chunk[:, :, r0:r0 + lens[j]]
+            self.vpool[:, :, pid, :lens[j]] = v_chunk[:, :, r0:r0 + lens[j]]
+            if lens[j] < w.bs:
+                self.kpool[:, :, pid, lens[j]:] = 0
+                self.vpool[:, :, pid, lens[j]:] = 0
+        self.set_chunk_meta(t)
+
+    # ------------------------------------------------------------ the hot path
+    def score(self, t, pool_ids=None, stream=None):
+        w = self.w
+        pids = self.chunk_ids(t) if pool_ids is None else pool_ids
+        K.score_blocks(self.d, self.q, w.chunk_tokens, self.kpool, self.NB, self.blk_len, pids,
+                       pids.numel(), self.q_bar, self.k_bar, self.scores, self.mem, stream)
+
+    def update(self, cand_ids, cand_src, stream=None):
+        if self.P == 0 or cand_ids.numel() == 0:
+            return
+        K.update_memory(self.d, self.kpool, self.vpool, self.NB, self.blk_len, self.blk_pos,
+                        self.k_bar, self.P, self.w.n_sink, self.slot_src, self.slot_w, cand_ids,
+                        cand_src, cand_ids.numel(), self.mem, self.w.policy, self.ws, stream)
+
+    def select(self, t, stream=None):
+        w = self.w
+        win = self.window_ids(t)
+        K.select_local(self.d, self.scores, self.nQB, self.NB, win, win.numel(), w.k,
+                       self.mem_ids, self.P, self.blk_len, w.mask, t * w.chunk_tokens,
+                       self.blk_pos, w.chunk_tokens, self.idx, self.cnt, self.Amax, 0, self.nQB,
+                       stream)
+
+    def attend(self, t, stream=None):
+        w = self.w
+        if self.tdtype == torch.bfloat16:
+            q, kp, vp = self.q, self.kpool, self.vpool
+        else:
+            self.q16.copy_(self.q)
+            self.k16.copy_(self.kpool)
+            self.v16.copy_(self.vpool)
+            q, kp, vp = self.q16, self.k16, self.v16
+        K.attn_fwd(self.dbf, q, w.chunk_tokens, t * w.chunk_tokens, kp, vp, self.NB, self.blk_len,
+                   self.blk_pos, self.idx, self.cnt, self.Amax, w.mask, self.o, self.lse, stream)
+
+    def candidates(self, t):
+        """Blocks that leave the window when chunk t arrives (rollout) or every
+        block older than the window (snapshot)."""
+        w = self.w
+        if w.rollout:
+            c = w.leaving_chunk(t)
+            chunks = [] if c is None else [c]
+        else:
+            chunks = w.snapshot_candidate_chunks()
+        key = ("cand",) + tuple(chunks) if not w.rollout else ("cand", t)
+        ci = self.ids(key + ("phys",), [p for c in chunks for p in w.chunk_phys_ids(c)])
+        cs = self.ids(key + ("src",), [g for c in chunks for g in w.chunk_global_ids(c)])
+        return ci, cs
+
+    def step(self, t, stream=None):
+        """Score -> update -> select -> attend for chunk t (its Q already in self.q,
+        its K/V already in the pool)."""
+        self.score(t, stream=stream)
+        ci, cs = self.candidates(t)
+        self.update(ci, cs, stream=stream)
+        self.select(t, stream=stream)
+        self.attend(t, stream=stream)

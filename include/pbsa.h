@@ -1,0 +1,240 @@
+/*
+ * pbsa.h -- C ABI of the PBSA (Persistent Block-Sparse Attention) hot path on
+ * NVIDIA B200 (sm_100a).
+ *
+ * Source of the operations: "Sparse Forcing: Native Trainable Sparse
+ * Attention for Real-time Autoregressive Diffusion Video Generation"
+ * (arXiv 2604.21221), as summarised on gist.science/es (section 2
+ * "Metodología: Sparse Forcing": items "Arquitectura Propuesta" and
+ * "Persistente Block-Sparse Attention (PBSA)") and in the paper's abstract
+ * (shd-paper.top page).  The pages describe the method in words only; the
+ * concrete formulas below are the plainest reading of them.
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ *  - All tensor arguments are DEVICE pointers owned by the caller; the library
+ *    allocates no device memory.  The only library-owned device state is one
+ *    status word per device (a __device__ variable, see pbsa_get_status).
+ *  - `stream` is a cudaStream_t passed as void*.  Every call is asynchronous
+ *    on that stream; nothing synchronises except pbsa_get_status.
+ *  - Batch-major layouts, all contiguous:
+ *      q, o, dO          [B, H, Tq, D]          (query chunk, Tq tokens)
+ *      kpool, vpool      [B, H, NB, bs, D]      (block pool, NB physical blocks)
+ *      blk_len, blk_pos  [B, H, NB]   int32     (valid rows of a block; global
+ *                                               token position of its row 0)
+ *      k_bar             [B, H, NB, D] float    (pooled key of each block)
+ *      q_bar             [B, H, nQB, D] float   nQB = ceil(Tq / bs)
+ *      scores            [B, H, nQB, NB] float
+ *      mem_score         [B, H, NB] float
+ *      slot_src, slot_w  [B, H, P]    int32 / float  (persistent slots are
+ *                                               physical ids 0..P-1)
+ *      idx               [B, H, nQB, Amax] int32 (attended physical ids,
+ *                                               ascending, padded with -1)
+ *      cnt               [B, H, nQB]  int32
+ *  - Query block i covers rows [i*bs, min((i+1)*bs, Tq)); a chunk is tiled on
+ *    its own, so its last block may be partial.  Rows of a block at or past
+ *    blk_len are padding: never read as tokens.
+ *  - Supported shapes: D in {64, 128}; bs in {64, 128}; B*H >= 1.
+ *  - bf16 buffers must be 16-byte aligned (128-bit loads and TMA); float and
+ *    int buffers 4-byte aligned.
+ *
+ * Errors
+ * ------
+ *  Every call validates its arguments on the host first and returns a negative
+ *  pbsa_status without launching anything when they are wrong.  A failed launch
+ *  returns PBSA_ERR_CUDA.  Faults found on the device (a bounded wait that ran
+ *  out) set the device status word, read and cleared by pbsa_get_status.
+ *  pbsa_last_error() gives a message for the last failing call of the thread.
+ */
+#ifndef PBSA_H
+#define PBSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  PBSA_OK = 0,
+  PBSA_ERR_ARG = -1,        /* null pointer, negative size, bad enum        */
+  PBSA_ERR_SHAPE = -2,      /* unsupported or inconsistent shape            */
+  PBSA_ERR_ALIGN = -3,      /* misaligned buffer                           */
+  PBSA_ERR_DTYPE = -4,      /* dtype not supported by this call            */
+  PBSA_ERR_CUDA = -5,       /* CUDA runtime error (launch, copy)           */
+  PBSA_ERR_TIMEOUT = -6,    /* device: a bounded wait ran out              */
+  PBSA_ERR_WORKSPACE = -7   /* workspace missing or too small              */
+} pbsa_status;
+
+typedef enum { PBSA_BF16 = 0, PBSA_FP32 = 1 } pbsa_dtype;
+typedef enum { PBSA_EVICT = 0, PBSA_MERGE_MEAN = 1 } pbsa_policy;
+typedef enum { PBSA_MASK_CHUNK = 0, PBSA_MASK_TOKEN = 1 } pbsa_mask;
+
+/* Problem dimensions shared by all calls.  scale multiplies <q, k> (usually
+ * 1/sqrt(D)); dtype is the storage type of q, kpool and vpool. */
+typedef struct {
+  int B, H, D, bs;
+  float scale;
+  int dtype; /* pbsa_dtype */
+} pbsa_dims;
+
+/* ---------------------------------------------------------------------------
+ * a1 + a2: block compression by pooling and coarse block scoring.
+ * Passage: gist.science/es section 2, PBSA item "Compresión de Bloques" (pooled
+ * block representatives for coarse routing) and item "Bloques Dinámicos"
+ * (coarse scoring of historical blocks for the current step).
+ *
+ *   q_bar[b,h,i]     = mean of the rows of query block i
+ *   k_bar[b,h,j]     = mean of the first blk_len[b,h,j] rows of block j, for
+ *                      j in pool_ids only (other entries are left as they are;
+ *                      a block of length 0 pools to zero)
+ *   scores[b,h,i,j]  = scale * <q_bar[b,h,i], k_bar[b,h,j]>  for all j < NB
+ *   mem_score[b,h,j] = mean over i of scores[b,h,i,j]
+ *
+ * q, kpool: dtype of dims (bf16 or fp32).  pool_ids: device int32 [n_pool],
+ * the same list for every (b,h); n_pool may be 0.  Outputs are overwritten.
+ * ------------------------------------------------------------------------- */
+int pbsa_score_blocks(const pbsa_dims* dims, const void* q, int Tq,
+                      const void* kpool, int NB, const int32_t* blk_len,
+                      const int32_t* pool_ids, int n_pool,
+                      float* q_bar, float* k_bar, float* scores, float* mem_score,
+                      void* stream);
+
+/* ---------------------------------------------------------------------------
+ * a3: persistent-memory update (Top-C retention, sinks, evict or mean-merge).
+ * Passage: gist.science/es section 2 "Arquitectura Propuesta", items "Memoria
+ * Persistente", "Bloques Sumidero", "Bloques Dinámicos", "Mecanismo de
+ * Actualización"; the abstract (the memory compresses as well as keeps its
+ * blocks); PBSA item "Optimización" (selective cache updates).
+ *
+ * Per (b,h): the candidates are the occupied non-sink slots (slot_src >= 0,
+ * index >= n_sink) and the blocks leaving the window, cand_ids (physical ids)
+ * with global ids cand_src.  A leaving block with cand_src < n_sink fills
+ * sink slot cand_src and is not ranked.  Candidates are ranked by
+ * mem_score (descending; ties: lower global id first) and the best
+ * P - n_sink are kept.  Kept slots stay where they are; newly kept blocks
+ * fill the free non-sink slots in ascending order, in ascending global-id
+ * order.  Losers are dropped (PBSA_EVICT) or, with PBSA_MERGE_MEAN, merged
+ * into the kept slot whose pre-merge pooled key has the largest dot product
+ * with theirs (ties: lowest slot).  A merged slot holds the weight-averaged,
+ * row-wise mean of its blocks (rows past a block's length count as zero),
+ * its weight is the sum of weights, its length the maximum, and its k_bar is
+ * the mean of its stored rows.  Slot rows, blk_len, blk_pos, k_bar, slot_src
+ * and slot_w of slot ids 0..P-1 are updated IN PLACE; other ids are only read.
+ *
+ * cand_ids, cand_src: device int32 [n_cand], same for every (b,h).
+ * Limits: 1 <= P <= 256, 0 <= n_sink <= P, (P - n_sink) + n_cand <= 256.
+ * workspace: device buffer of at least pbsa_update_memory_workspace() bytes,
+ * 256-byte aligned; its contents need not be initialised.
+ * ------------------------------------------------------------------------- */
+size_t pbsa_update_memory_workspace(const pbsa_dims* dims, int P, int n_cand);
+int pbsa_update_memory(const pbsa_dims* dims, void* kpool, void* vpool, int NB,
+                       int32_t* blk_len, int32_t* blk_pos, float* k_bar,
+                       int P, int n_sink, int32_t* slot_src, float* slot_w,
+                       const int32_t* cand_ids, const int32_t* cand_src, int n_cand,
+                       const float* mem_score, int policy,
+                       void* workspace, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * a4 + a5: local Top-K selection and the attended-block list.
+ * Passage: gist.science/es section 2 "Arquitectura Propuesta", item "Ventana
+ * Local" (per-query Top-K of relevant blocks inside the sliding window) and
+ * PBSA item "Atención Híbrida" (dense over the persistent memory).
+ *
+ * For each (b,h) and query block i < nQB of this call:
+ *   candidates = win_ids[0..n_win) with blk_len > 0 (and, with PBSA_MASK_TOKEN,
+ *                blk_pos <= q_pos0 + last row of block i);
+ *   local      = the best min(k, #candidates) by scores[b,h,i,j] (descending;
+ *                ties: lower physical id first);
+ *   list       = mem_ids[b,h,0..n_mem) entries >= 0 with blk_len > 0, united
+ *                with local, ascending, without duplicates.
+ * Written to idx[b,h,qb_offset+i,0..cnt) (rest -1) and cnt[b,h,qb_offset+i],
+ * where idx/cnt have nQB_total query-block rows.
+ *
+ * scores: [B,H,nQB,NB] float, indexed by the same physical ids as blk_len
+ * and blk_pos [B,H,NB].  win_ids: device int32 [n_win], same for every
+ * (b,h).  mem_ids: device int32 [B,H,n_mem] or NULL with n_mem = 0.
+ * blk_pos may be NULL with PBSA_MASK_CHUNK.  Tq is this call's query rows
+ * (used for the token mask).  Limits: n_win <= 256, n_mem + min(k, n_win) <=
+ * min(Amax, 256).
+ * ------------------------------------------------------------------------- */
+int pbsa_select_local(const pbsa_dims* dims, const float* scores, int nQB, int NB,
+                      const int32_t* win_ids, int n_win, int k,
+                      const int32_t* mem_ids, int n_mem,
+                      const int32_t* blk_len, int mask, int q_pos0, const int32_t* blk_pos,
+                      int Tq, int32_t* idx, int32_t* cnt, int Amax,
+                      int qb_offset, int nQB_total, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * a6: hybrid block-sparse attention, forward.
+ * Passage: gist.science/es section 2 PBSA item "Atención Híbrida" (dense over
+ * the persistent memory plus sparse over the local window, one kernel) and
+ * item "Optimización" (irregular sparsity); section 4 (speed-up over
+ * FlashAttention-2 grows with sparsity).
+ *
+ * For each row r of query block i: one softmax over the valid rows of the
+ * blocks idx[b,h,i,0..cnt):
+ *   O[r]   = sum_c softmax_c(scale * <q_r, k_c>) v_c
+ *   lse[r] = log sum_c exp(scale * <q_r, k_c>)          (natural log)
+ * PBSA_MASK_TOKEN keeps only keys with blk_pos + row <= q_pos0 + r.  A row
+ * with no visible key gets O = 0 and lse = -inf.
+ * q, kpool, vpool, o: bf16 only (dims.dtype must be PBSA_BF16); lse: float.
+ * Every idx entry must be in [0, NB); cnt <= Amax.  Runs on tcgen05 tensor
+ * cores (sm_100a).
+ * ------------------------------------------------------------------------- */
+int pbsa_attn_fwd(const pbsa_dims* dims, const void* q, int Tq, int q_pos0,
+                  const void* kpool, const void* vpool, int NB,
+                  const int32_t* blk_len, const int32_t* blk_pos,
+                  const int32_t* idx, const int32_t* cnt, int Amax, int mask,
+                  void* o, float* lse, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * a7: backward of pbsa_attn_fwd for the trainable path.
+ * Passage: gist.science/es section 2 "Entrenamiento" (training with the
+ * dynamically updated cache) and section 3 "Contribuciones Clave", item
+ * "Kernel PBSA" (the kernel serves training as well as inference).
+ *
+ * The attended lists are constants.  With P the forward's softmax:
+ *   dV_c += P^T dO,  dP = dO V^T,  Delta_r = <dO_r, O_r>,
+ *   dS = P * (dP - Delta),  dQ = scale * dS K,  dK_c += scale * dS^T Q.
+ * o, lse are the forward's outputs; dO bf16 [B,H,Tq,D].  dq [B,H,Tq,D],
+ * dk/dv [B,H,NB,bs,D] are float and fully overwritten (blocks nobody attends
+ * get zero).  workspace: at least pbsa_attn_bwd_workspace() bytes.
+ * ------------------------------------------------------------------------- */
+size_t pbsa_attn_bwd_workspace(const pbsa_dims* dims, int Tq, int NB, int Amax);
+int pbsa_attn_bwd(const pbsa_dims* dims, const void* q, int Tq, int q_pos0,
+                  const void* kpool, const void* vpool, int NB,
+                  const int32_t* blk_len, const int32_t* blk_pos,
+                  const int32_t* idx, const int32_t* cnt, int Amax, int mask,
+                  const void* o, const float* lse, const void* dO,
+                  float* dq, float* dk, float* dv,
+                  void* workspace, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Status and diagnostics (no counterpart on the pages).
+ * ------------------------------------------------------------------------- */
+
+/* Synchronises `stream`, returns the device status word of the current device
+ * (PBSA_OK, or PBSA_ERR_TIMEOUT when a kernel's bounded wait ran out) and
+ * clears it.  Returns PBSA_ERR_CUDA if the read itself fails. */
+int pbsa_get_status(void* stream);
+
+/* Message for the last failing call made by this host thread ("" if none). */
+const char* pbsa_last_error(void);
+
+/* Library version string. */
+const char* pbsa_version(void);
+
+/* Test hook for the failure path.  Sets the time limit of every bounded
+ * device wait (nanoseconds; <= 0 restores the default of 2 s) and debug
+ * flags: bit 0 makes the next pbsa_attn_fwd launches skip the first V-tile
+ * load, so that the tensor-core issuer's wait for it runs out, the kernel
+ * sets PBSA_ERR_TIMEOUT and every CTA returns cleanly. */
+void pbsa_set_debug(int flags, int64_t wait_limit_ns);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PBSA_H */

@@ -397,6 +397,20 @@ def _logits(qi, kc, scale, mask, q_rows_pos, k_pos):
     return s
 
 
+def _softmax_rows(s):
+    """Row-wise softmax of logits s [n, keys] and its log-normaliser.
+
+    A row whose logits are all -inf (no visible key) gets P = 0, LSE = -inf."""
+    has = np.isfinite(s).any(axis=1)
+    mx = np.where(has, np.max(np.where(np.isfinite(s), s, -np.inf), axis=1, initial=-np.inf), 0.0)
+    mx = np.where(has, mx, 0.0)
+    e = np.exp(s - mx[:, None])
+    z = e.sum(axis=1)
+    P = np.where(has[:, None], e / np.where(has, z, 1.0)[:, None], 0.0)
+    lse = np.where(has, mx + np.log(np.where(has, z, 1.0)), -np.inf)
+    return P, lse
+
+
 def attention_fwd(q, kpool, vpool, blk_len, blk_pos, idx, cnt, scale: float,
                   mask: int = MASK_CHUNK, q_pos0: int = 0):
     """One softmax over the union of the attended blocks of each query block (R12).
@@ -422,15 +436,9 @@ def attention_fwd(q, kpool, vpool, blk_len, blk_pos, idx, cnt, scale: float,
                     continue
                 qi = q[b, h, r0:r0 + n].astype(np.float64)
                 s = _logits(qi, kc, scale, mask, q_pos0 + r0 + np.arange(n), kpos)
-                for r in range(n):
-                    row = s[r]
-                    if not np.isfinite(row).any():
-                        continue
-                    mx = row.max()
-                    e = np.exp(row - mx)
-                    z = e.sum()
-                    O[b, h, r0 + r] = (e / z) @ vc
-                    LSE[b, h, r0 + r] = mx + math.log(z)
+                P, lse = _softmax_rows(s)
+                O[b, h, r0:r0 + n] = P @ vc
+                LSE[b, h, r0:r0 + n] = lse
     return O, LSE
 
 
@@ -464,11 +472,7 @@ def attention_bwd(q, kpool, vpool, blk_len, blk_pos, idx, cnt, dO, scale: float,
                 qi = q[b, h, r0:r0 + n].astype(np.float64)
                 doi = dO[b, h, r0:r0 + n].astype(np.float64)
                 s = _logits(qi, kc, scale, mask, q_pos0 + r0 + np.arange(n), kpos)
-                Pm = np.zeros_like(s)
-                for r in range(n):
-                    if np.isfinite(s[r]).any():
-                        e = np.exp(s[r] - s[r].max())
-                        Pm[r] = e / e.sum()
+                Pm, _ = _softmax_rows(s)
                 dvc = Pm.T @ doi
                 dP = doi @ vc.T
                 dS = Pm * (dP - (Pm * dP).sum(axis=1, keepdims=True))
