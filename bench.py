@@ -1,0 +1,450 @@
+#!/usr/bin/env python
+"""Benchmark of the PBSA hot path on B200.
+
+Default workload (N=1): one single-layer decode step shaped like a 1.3B video
+DiT -- B1 H12 D128 bf16, 128-token blocks, a 4680-token query chunk (37
+blocks), a cache of 5 chunks (185 blocks), persistent budget 24, window of 2
+chunks, local top-16 -- run as score -> update memory -> select -> attend.
+A step is one pass of that path over the chunk; the memory starts empty each
+step (snapshot semantics) and the pooled keys of older blocks are cached, so
+the step pools only the current chunk's Q and K.
+
+Reported (one JSON line on rank 0):
+  value          attended forward TFLOP/s over the whole step (all ranks)
+  ms_per_step    per-chunk latency of the step (device time, max over ranks)
+  roofline       the attention kernel against the measured bf16 peak
+  e2e            the same metric through the public API with pinned host
+                 inputs copied in and the output copied out every step
+  cpu_baseline   the CPU oracle timed on a bounded sample on the host cores
+  --impl reference  times the CPU oracle itself as the reference arm.
+
+Multi-GPU (torchrun): every rank runs its own decode problem (independent
+layers/sequences), no data-path collective; scaling is weak.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_FLUSH_BYTES = 256 << 20
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="pbsa", choices=["pbsa", "reference"])
+    ap.add_argument("--workload", default="decode", choices=["decode"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    return ap.parse_args()
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+# ----------------------------------------------------------------- distributed
+def init_dist(n):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ----------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.15)
+        self.proc.terminate()
+        out, _ = self.proc.communicate(timeout=10)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": float(np.median(sm)) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------- decode
+class DecodeRunner:
+    """One decode-step problem resident on the device, captured as a CUDA graph."""
+
+    def __init__(self, seed_offset=0):
+        import torch
+
+        import pbsa_inputs as PI
+        from block_sparse_attention_39_b200.engine import PbsaLayer
+        self.torch = torch
+        w = PI.WORKLOADS["decode"]
+        if seed_offset:
+            w = PI.variant(w, seed=w.seed + 1000 * seed_offset)
+        self.w = w
+        snap = PI.snapshot(w)
+        self.snap = snap
+        L = PbsaLayer(w)
+        dev = torch.device("cuda")
+
+        def st(x):
+            return torch.from_numpy(np.ascontiguousarray(x)).to(dev).to(torch.bfloat16)
+        L.kpool.copy_(st(snap["kpool"]))
+        L.vpool.copy_(st(snap["vpool"]))
+        L.blk_len.copy_(torch.from_numpy(snap["blk_len"]).to(dev))
+        L.blk_pos.copy_(torch.from_numpy(snap["blk_pos"]).to(dev))
+        L.q.copy_(st(snap["q"]))
+        self.L = L
+        self.t = w.n_chunks - 1
+        # pooled keys of every cached block (older blocks stay cached)
+        L.score(self.t, pool_ids=L.ids(("all",), snap["all_ids"]))
+        L.reset_memory()
+        self.cand = L.candidates(self.t)
+        L.window_ids(self.t)
+        L.chunk_ids(self.t)
+        torch.cuda.synchronize()
+        self.flush_buf = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+        self.launches_per_step = 6   # pool, score, plan, apply, select, attention
+
+    def step(self, ev=None):
+        L = self.L
+        if ev is not None:
+            ev[0].record()
+        L.score(self.t)
+        if ev is not None:
+            ev[1].record()
+        L.update(*self.cand)
+        if ev is not None:
+            ev[2].record()
+        L.select(self.t)
+        if ev is not None:
+            ev[3].record()
+        L.attend(self.t)
+        if ev is not None:
+            ev[4].record()
+
+    def prologue(self):
+        self.L.reset_memory()
+        self.flush_buf.zero_()
+
+    def flops(self):
+        L = self.L
+        idx = L.idx.cpu().numpy()
+        cnt = L.cnt.cpu().numpy()
+        bl = L.blk_len.cpu().numpy()
+        lens = np.array(self.w.chunk_block_lens(), dtype=np.int64)
+        total = 0
+        for b in range(self.w.B):
+            for h in range(self.w.H):
+                for i in range(L.nQB):
+                    ids = idx[b, h, i, :cnt[b, h, i]]
+                    total += 4 * int(lens[i]) * int(bl[b, h, ids].astype(np.int64).sum()) * self.w.D
+        return total
+
+    def capture(self, n_graphs):
+        """Capture n_graphs copies of [prologue, e0, score, e1, update, e2, select, e3,
+        attend, e4], each with its own timing events (event-record graph nodes)."""
+        torch = self.torch
+        s = torch.cuda.Stream()
+        torch.cuda.synchronize()
+        with torch.cuda.stream(s):
+            for _ in range(3):                   # eager warm-up before capture
+                self.prologue()
+                self.step()
+        torch.cuda.synchronize()
+        pool = torch.cuda.graph_pool_handle()
+        graphs, evs = [], []
+        for _ in range(n_graphs):
+            ev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(5)]
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, pool=pool, stream=s):
+                self.prologue()
+                self.step(ev)
+            graphs.append(g)
+            evs.append(ev)
+        torch.cuda.synchronize()
+        return graphs, evs, s
+
+    def e2e(self, steps, warmup):
+        """Through the public API with host buffers: pinned Q and new-chunk K/V in,
+        O and LSE out, every step."""
+        torch = self.torch
+        L, w = self.L, self.w
+        ids = w.chunk_phys_ids(self.t)
+        p0, p1 = ids[0], ids[-1] + 1
+        hq = torch.from_numpy(self.snap["q"]).to(torch.bfloat16).pin_memory()
+        hk = torch.from_numpy(np.ascontiguousarray(self.snap["kpool"][:, :, p0:p1])).to(
+            torch.bfloat16).pin_memory()
+        hv = torch.from_numpy(np.ascontiguousarray(self.snap["vpool"][:, :, p0:p1])).to(
+            torch.bfloat16).pin_memory()
+        ho = torch.empty(L.o.shape, dtype=torch.bfloat16).pin_memory()
+        hl = torch.empty(L.lse.shape, dtype=torch.float32).pin_memory()
+        dk = L.kpool[:, :, p0:p1]
+        dv = L.vpool[:, :, p0:p1]
+        h2d = hq.numel() * 2 + hk.numel() * 2 + hv.numel() * 2
+        d2h = ho.numel() * 2 + hl.numel() * 4
+        s = torch.cuda.Stream()
+        times = []
+        with torch.cuda.stream(s):
+            for it in range(warmup + steps):
+                self.prologue()
+                e0 = torch.cuda.Event(enable_timing=True)
+                e1 = torch.cuda.Event(enable_timing=True)
+                e0.record(s)
+                L.q.copy_(hq, non_blocking=True)
+                dk.copy_(hk, non_blocking=True)
+                dv.copy_(hv, non_blocking=True)
+                self.step()
+                ho.copy_(L.o, non_blocking=True)
+                hl.copy_(L.lse, non_blocking=True)
+                e1.record(s)
+                if it >= warmup:
+                    times.append((e0, e1))
+        torch.cuda.synchronize()
+        ms = float(np.mean([a.elapsed_time(b) for a, b in times]))
+        return ms, h2d, d2h
+
+
+# ----------------------------------------------------------------- CPU oracle
+def cpu_oracle_sample(w, snap, n_heads=2, n_qblocks=None):
+    """Time the oracle on a bounded sample: the full score/update/select on the
+    sampled heads plus attention on their query blocks.  Returns
+    (attended FLOPs of the sample, seconds, description)."""
+    import oracle as O
+    import pbsa_inputs as PI
+    H = n_heads
+    sub = {k: (v[:, :H] if isinstance(v, np.ndarray) and v.ndim >= 3 and v.shape[1] == w.H else v)
+           for k, v in snap.items()}
+    ws = PI.variant(w, H=H)
+    t0 = time.perf_counter()
+    kp = sub["kpool"].astype(np.float64)
+    vp = sub["vpool"].astype(np.float64)
+    kb0 = np.zeros((w.B, H, w.NB_phys, w.D))
+    qb, kb, S, m = O.score_blocks(sub["q"], kp, sub["blk_len"], sub["all_ids"], kb0, w.scale, w.bs)
+    up = O.update_memory(kp, vp, sub["blk_len"], sub["blk_pos"], kb, sub["slot_src"],
+                         sub["slot_w"], sub["cand_ids"], sub["cand_src"], m, w.P, w.n_sink,
+                         w.policy, w.dtype)
+    kp2, vp2, bl2, bp2 = up[0], up[1], up[2], up[3]
+    A = O.select_local(S, sub["win_ids"], w.k, PI.mem_ids_all_slots(ws), bl2, w.mask,
+                       sub["q_pos0"], bp2, w.bs, w.chunk_tokens)
+    idx, cnt = O.lists_to_arrays(A, PI.amax(w))
+    nq = idx.shape[2] if n_qblocks is None else n_qblocks
+    q = sub["q"][:, :, :nq * w.bs]
+    O.attention_fwd(q, kp2, vp2, bl2, bp2, idx[:, :, :nq], cnt[:, :, :nq], w.scale, w.mask,
+                    sub["q_pos0"])
+    dt = time.perf_counter() - t0
+    lens = np.array(w.chunk_block_lens(), dtype=np.int64)
+    fl = 0
+    for h in range(H):
+        for i in range(nq):
+            ids = idx[0, h, i, :cnt[0, h, i]]
+            fl += 4 * int(lens[i]) * int(bl2[0, h, ids].astype(np.int64).sum()) * w.D
+    return fl, dt, f"{H} of {w.H} heads, {nq} of {idx.shape[2]} query blocks, full score/update/select"
+
+
+def cores_used():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count()
+
+
+def config_of(w):
+    return {"workload": (f"decode step: B{w.B} H{w.H} D{w.D} bf16, {w.bs}-token blocks, "
+                         f"query chunk {w.chunk_tokens} tokens ({w.nb_c} blocks), cache "
+                         f"{w.n_chunks} chunks ({w.n_chunks * w.nb_c} blocks), P{w.P} "
+                         f"W{w.W} chunks k{w.k}, evict"),
+            "global_batch": w.B, "seq_len": w.chunk_tokens,
+            "cache_tokens": w.n_chunks * w.chunk_tokens,
+            "l2": "flushed between steps (256 MiB device write outside the timed events)",
+            "parallelism": "replicas"}
+
+
+# ----------------------------------------------------------------- main
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+    import torch
+    rank, world, local = init_dist(args.gpus)
+    pk, pk_kind = peaks()
+    runner = DecodeRunner(seed_offset=rank)
+    w = runner.w
+    n_graphs = max(1, min(64, args.steps))
+    graphs, evs, s = runner.capture(n_graphs)
+    with torch.cuda.stream(s):
+        for i in range(args.warmup):
+            graphs[i % n_graphs].replay()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local)
+    barrier(world)
+    torch.cuda.synchronize()
+    clocks.start()
+    wall0 = time.perf_counter()
+    rows = []
+    done = 0
+    while done < args.steps:
+        n = min(n_graphs, args.steps - done)
+        with torch.cuda.stream(s):
+            for i in range(n):
+                graphs[i].replay()
+        torch.cuda.synchronize()
+        rows += [[evs[i][k].elapsed_time(evs[i][k + 1]) for k in range(4)] for i in range(n)]
+        done += n
+    wall = time.perf_counter() - wall0
+    barrier(world)
+    clk = clocks.stop()
+    per = np.array(rows)                  # ms: score, update, select, attention
+    step_ms = per.sum(axis=1)
+    ms_step = float(step_ms.mean())
+    ms_attn = float(per[:, 3].mean())
+    ms_step_max = max_over_ranks(ms_step, world)
+    flops = runner.flops()
+    value = world * flops / (ms_step_max * 1e-3) / 1e12
+    attn_tflops = flops / (ms_attn * 1e-3) / 1e12
+    peak = pk["bf16_tflops"]
+    # HBM view of the HBM-bound calls: algorithmic bytes of score (read Q chunk +
+    # new K blocks, write q_bar/k_bar/scores/mem) and of the update (copy 24 blocks)
+    line = {
+        "metric": "PBSA fwd effective TFLOP/s (attended blocks) & per-chunk latency",
+        "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_step_max, 5), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) Q/K/V, salience offsets N(0,2) on 10% of key blocks)",
+        "config": config_of(w),
+        "per_call_ms": {"score_blocks": round(float(per[:, 0].mean()), 5),
+                        "update_memory": round(float(per[:, 1].mean()), 5),
+                        "select_local": round(float(per[:, 2].mean()), 5),
+                        "attn_fwd": round(ms_attn, 5)},
+        "attended_gflop_per_step": round(flops / 1e9, 3),
+        "roofline": {"kernel": "attn_fwd_kernel<128,128,3,2>", "bound": "tensor",
+                     "achieved": round(attn_tflops, 2), "peak": peak, "unit": "TFLOP/s",
+                     "frac": round(attn_tflops / peak, 4), "traffic": None,
+                     "peak_kind": f"bf16_tflops burst, {pk_kind}"},
+        "gpu_launches": runner.launches_per_step * args.steps,
+        "clocks": clk,
+        "wall_s_timed_region": round(wall, 3),
+    }
+    if not args.no_e2e:
+        e2e_ms, h2d, d2h = runner.e2e(steps=min(args.steps, 50), warmup=5)
+        e2e_ms = max_over_ranks(e2e_ms, world)
+        line["e2e"] = {"value": round(world * flops / (e2e_ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+                       "ms_per_step": round(e2e_ms, 4), "h2d_bytes_per_step": h2d,
+                       "d2h_bytes_per_step": d2h}
+    if rank == 0 and not args.no_cpu:
+        fl, dt, desc = cpu_oracle_sample(w, runner.snap)
+        line["cpu_baseline"] = {"value": round(fl / dt / 1e12, 6), "unit": "TFLOP/s",
+                                "cores": cores_used(), "kind": "oracle", "sample": desc,
+                                "seconds": round(dt, 2)}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        del graphs
+        dist.destroy_process_group()
+
+
+def run_reference(args):
+    """Reference arm: the CPU oracle, as it stands, on the host cores."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import pbsa_inputs as PI
+    w = PI.WORKLOADS["decode"]
+    snap = PI.snapshot(w)
+    times, fls = [], []
+    desc = ""
+    # keep the whole run to a few minutes: smaller samples when many steps are asked
+    nq = 8 if args.warmup + args.steps <= 100 else 1
+    for it in range(args.warmup + args.steps):
+        fl, dt, desc = cpu_oracle_sample(w, snap, n_heads=1, n_qblocks=nq)
+        if it >= args.warmup:
+            times.append(dt)
+            fls.append(fl)
+    ms = float(np.mean(times)) * 1e3
+    value = float(np.mean(fls)) / (ms * 1e-3) / 1e12
+    line = {"impl": "reference", "metric": "PBSA fwd effective TFLOP/s (attended blocks) & per-chunk latency",
+            "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(ms, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": config_of(w),
+            "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": cores_used(),
+                             "kind": "oracle", "sample": "each step: " + desc},
+            "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -17,7 +17,7 @@ c_int, c_float, c_void_p, c_size_t, c_int64 = (ctypes.c_int, ctypes.c_float, cty
 
 class PbsaDims(ctypes.Structure):
     _fields_ = [("B", c_int), ("H", c_int), ("D", c_int), ("bs", c_int), ("scale", c_float),
-                ("dtype", c_int)]
+                ("dtype", c_int), ("q_chunk", c_int)]
 
 
 P = ctypes.POINTER(PbsaDims)

@@ -6,15 +6,17 @@
 // "Optimización").  Here both parts are one list of physical block ids per
 // query block, and one softmax runs over their union.
 //
-// Design (one CTA per 128-row query tile, 6 warps):
-//   warp 4      TMA producer: Q tile once, then K_j / V_j of every listed
-//               block j, gathered by row coordinate from the block pool,
-//               through an NST-stage shared-memory ring (128-byte swizzle);
-//               also allocates / frees tensor memory;
-//   warp 5      tcgen05 issuer (one thread): S_j = Q K_j^T into one of two
-//               TMEM score buffers, then O += P_j V_j with P_j read from TMEM;
-//               QK_{j+1} is issued before waiting for P_j so the tensor core
-//               works while the softmax warps handle block j;
+// Design (one CTA per 128-row query tile, 7 warps):
+//   warp 4      TMA producer of the Q tile and of K_j for every listed block j,
+//               gathered by row coordinate from the block pool through an
+//               NSK-stage ring (128-byte swizzle); a K stage is released as
+//               soon as its QK^T has run; also allocates / frees TMEM;
+//   warp 6      TMA producer of V_j through an NSV-stage ring;
+//   warp 5      tcgen05 issuer (one thread): S_0, S_1 first; then for each j,
+//               O += P_j V_j (P_j read from TMEM) as soon as the softmax has
+//               written it, followed by S_{j+2} = Q K_{j+2}^T into the score
+//               buffer just freed -- so the tensor core runs PV_j and QK_{j+2}
+//               while the softmax warps handle block j+1;
 //   warps 0-3   softmax (thread = query row = TMEM lane): fp32 online softmax
 //               in the log2 domain with a lazily moved reference maximum
 //               (O in TMEM is rescaled only when the row maximum grows by
@@ -43,14 +45,14 @@ struct FwdParams {
   const int32_t* cnt;
   __nv_bfloat16* o;
   float* lse;
-  int B, H, Tq, q_pos0, NB, Amax, nQB, mask;
+  int B, H, Tq, q_chunk, q_pos0, NB, Amax, nQB, mask;
   float scale_log2;
   int* status;
   int64_t limit_ns;
   int debug;
 };
 
-template <int D, int BS, int NST>
+template <int D, int BS, int NSK, int NSV>
 struct FwdCfg {
   static constexpr int BM = 128;
   static constexpr int KB = D / 64;            // 64-column (128-byte) boxes per row
@@ -60,18 +62,19 @@ struct FwdCfg {
   static constexpr int KV_BYTES = KB * BOX_KV;
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + Q_BYTES;
-  static constexpr int OFF_V = OFF_K + NST * KV_BYTES;
-  static constexpr int OFF_BAR = OFF_V + NST * KV_BYTES;
+  static constexpr int OFF_V = OFF_K + NSK * KV_BYTES;
+  static constexpr int OFF_BAR = OFF_V + NSV * KV_BYTES;
   // barrier indices
   static constexpr int B_Q = 0;
-  static constexpr int B_KF = 1;                 // + stage
-  static constexpr int B_VF = 1 + NST;           // + stage
-  static constexpr int B_KVE = 1 + 2 * NST;      // + stage
-  static constexpr int B_SF = 1 + 3 * NST;       // + buffer (2)
-  static constexpr int B_PF = 3 + 3 * NST;       // + buffer (2)
-  static constexpr int B_OD = 5 + 3 * NST;       // + buffer (2)
-  static constexpr int B_MMA = 7 + 3 * NST;
-  static constexpr int NBAR = 8 + 3 * NST;
+  static constexpr int B_KF = 1;                         // + K stage
+  static constexpr int B_KE = B_KF + NSK;                // + K stage
+  static constexpr int B_VF = B_KE + NSK;                // + V stage
+  static constexpr int B_VE = B_VF + NSV;                // + V stage
+  static constexpr int B_SF = B_VE + NSV;                // + S buffer (2)
+  static constexpr int B_PF = B_SF + 2;                  // + P buffer (2)
+  static constexpr int B_OD = B_PF + 2;                  // + parity of the PV (2)
+  static constexpr int B_MMA = B_OD + 2;
+  static constexpr int NBAR = B_MMA + 1;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int OFF_IDS = OFF_MISC + 16;
   // tensor-memory columns
@@ -86,11 +89,15 @@ struct FwdCfg {
   static size_t smem_bytes(int Amax) { return 1024 + OFF_IDS + 3 * 4 * static_cast<size_t>(Amax); }
 };
 
-template <int D, int BS, int NST>
-__global__ void __launch_bounds__(192, 1)
+// Warp roles: 0-3 softmax / epilogue, 4 K producer + TMEM owner, 5 MMA issuer,
+// 6 V producer.
+constexpr int kFwdThreads = 224;
+
+template <int D, int BS, int NSK, int NSV>
+__global__ void __launch_bounds__(kFwdThreads, 1)
 attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                 const __grid_constant__ CUtensorMap tmV, FwdParams p) {
-  using C = FwdCfg<D, BS, NST>;
+  using C = FwdCfg<D, BS, NSK, NSV>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -103,7 +110,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     if (tid == 0) report_status(p.status, PBSA_ERR_ARG);
     n = n < 0 ? 0 : p.Amax;
   }
-  const int qlen = min(BS, p.Tq - qi * BS);
+  int qrow0, qlen;                  // first row and rows of this query block
+  qb_rows(qi, p.Tq, p.q_chunk, BS, qrow0, qlen);
 
   const uint32_t sQ = smem_u32(smem + C::OFF_Q);
   const uint32_t sK = smem_u32(smem + C::OFF_K);
@@ -118,10 +126,13 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
 
   if (tid == 0) {
     mbar_init(BAR(C::B_Q), 1);
-    for (int s = 0; s < NST; ++s) {
+    for (int s = 0; s < NSK; ++s) {
       mbar_init(BAR(C::B_KF + s), 1);
+      mbar_init(BAR(C::B_KE + s), 1);
+    }
+    for (int s = 0; s < NSV; ++s) {
       mbar_init(BAR(C::B_VF + s), 1);
-      mbar_init(BAR(C::B_KVE + s), 1);
+      mbar_init(BAR(C::B_VE + s), 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(BAR(C::B_SF + b), 1);
@@ -157,28 +168,48 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   const uint32_t tmem = *tmem_holder;
 
   if (warp == 4) {
-    // ------------------------------------------------------------ producer
+    // ------------------------------------------------------------ K producer
     if (lane == 0 && n > 0) {
       prefetch_tmap(&tmQ);
       prefetch_tmap(&tmK);
-      prefetch_tmap(&tmV);
-      const int q_row = bh * p.Tq + qi * BS;
+      const int q_row = bh * p.Tq + qrow0;
       mbar_expect_tx(BAR(C::B_Q), C::Q_BYTES);
 #pragma unroll
       for (int kb = 0; kb < C::KB; ++kb) tma_load_2d(sQ + kb * C::BOX_Q, &tmQ, BAR(C::B_Q), kb * 64, q_row);
       int issued = 0;
-      const bool skip_v0 = (p.debug & 1) != 0;
       for (int j = 0; j < n; ++j) {
-        const int s = j % NST;
-        if (j >= NST &&
-            !mbar_wait(BAR(C::B_KVE + s), ((j / NST) & 1) ^ 1, abort_flag, p.status, p.limit_ns))
+        const int s = j % NSK;
+        if (j >= NSK &&
+            !mbar_wait(BAR(C::B_KE + s), ((j / NSK) & 1) ^ 1, abort_flag, p.status, p.limit_ns))
           break;
         const int kv_row = (bh * p.NB + s_ids[j]) * BS;
         mbar_expect_tx(BAR(C::B_KF + s), C::KV_BYTES);
 #pragma unroll
         for (int kb = 0; kb < C::KB; ++kb)
           tma_load_2d(sK + s * C::KV_BYTES + kb * C::BOX_KV, &tmK, BAR(C::B_KF + s), kb * 64, kv_row);
+        issued = j + 1;
+      }
+      // no copy may still be in flight when the CTA leaves
+      mbar_drain(BAR(C::B_Q), 0, p.status, p.limit_ns);
+      for (int s = 0; s < NSK && s < issued; ++s) {
+        const int jl = s + ((issued - 1 - s) / NSK) * NSK;   // last load issued to stage s
+        mbar_drain(BAR(C::B_KF + s), (jl / NSK) & 1, p.status, p.limit_ns);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 6) {
+    // ------------------------------------------------------------ V producer
+    if (lane == 0 && n > 0) {
+      prefetch_tmap(&tmV);
+      const bool skip_v0 = (p.debug & 1) != 0;
+      int issued = 0;
+      for (int j = 0; j < n; ++j) {
+        const int s = j % NSV;
+        if (j >= NSV &&
+            !mbar_wait(BAR(C::B_VE + s), ((j / NSV) & 1) ^ 1, abort_flag, p.status, p.limit_ns))
+          break;
         if (!(skip_v0 && j == 0)) {
+          const int kv_row = (bh * p.NB + s_ids[j]) * BS;
           mbar_expect_tx(BAR(C::B_VF + s), C::KV_BYTES);
 #pragma unroll
           for (int kb = 0; kb < C::KB; ++kb)
@@ -187,12 +218,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         }
         issued = j + 1;
       }
-      // no copy may still be in flight when the CTA leaves
-      mbar_drain(BAR(C::B_Q), 0, p.status, p.limit_ns);
-      for (int s = 0; s < NST && s < issued; ++s) {
-        const int jl = s + ((issued - 1 - s) / NST) * NST;   // last load issued to stage s
-        mbar_drain(BAR(C::B_KF + s), (jl / NST) & 1, p.status, p.limit_ns);
-        if (!(skip_v0 && jl == 0)) mbar_drain(BAR(C::B_VF + s), (jl / NST) & 1, p.status, p.limit_ns);
+      for (int s = 0; s < NSV && s < issued; ++s) {
+        const int jl = s + ((issued - 1 - s) / NSV) * NSV;
+        if (!(skip_v0 && jl == 0)) mbar_drain(BAR(C::B_VF + s), (jl / NSV) & 1, p.status, p.limit_ns);
       }
     }
     __syncwarp();
@@ -201,9 +229,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     if (lane == 0 && n > 0) {
       constexpr uint32_t idesc_qk = idesc_bf16_f32(128, BS, false, false);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, false, true);
+      // S_j = Q K_j^T into S buffer (j & 1); frees K stage j % NSK when done
       auto issue_qk = [&](int j) -> bool {
-        const int s = j % NST;
-        if (!mbar_wait(BAR(C::B_KF + s), (j / NST) & 1, abort_flag, p.status, p.limit_ns))
+        const int s = j % NSK;
+        if (!mbar_wait(BAR(C::B_KF + s), (j / NSK) & 1, abort_flag, p.status, p.limit_ns))
           return false;
         tc_fence_after();
         const uint32_t d_tm = tmem + ((j & 1) ? C::TM_S1 : C::TM_S0);
@@ -216,25 +245,28 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           mma_ss(d_tm, a, b, idesc_qk, k > 0 ? 1u : 0u);
         }
         mma_commit(BAR(C::B_SF + (j & 1)));
+        mma_commit(BAR(C::B_KE + s));
         return true;
       };
-      if (mbar_wait(BAR(C::B_Q), 0, abort_flag, p.status, p.limit_ns) && issue_qk(0)) {
-        for (int j = 0; j < n; ++j) {
-          if (j + 1 < n && !issue_qk(j + 1)) break;
-          if (!mbar_wait(BAR(C::B_PF + (j & 1)), (j >> 1) & 1, abort_flag, p.status, p.limit_ns))
-            break;
-          const int s = j % NST;
-          if (!mbar_wait(BAR(C::B_VF + s), (j / NST) & 1, abort_flag, p.status, p.limit_ns)) break;
-          tc_fence_after();
-          const uint32_t p_tm = tmem + ((j & 1) ? C::TM_P1 : C::TM_P0);
+      bool ok = mbar_wait(BAR(C::B_Q), 0, abort_flag, p.status, p.limit_ns) && issue_qk(0) &&
+                (n < 2 || issue_qk(1));
+      for (int j = 0; ok && j < n; ++j) {
+        // O += P_j V_j once the softmax has written P_j
+        if (!mbar_wait(BAR(C::B_PF + (j & 1)), (j >> 1) & 1, abort_flag, p.status, p.limit_ns))
+          break;
+        const int sv = j % NSV;
+        if (!mbar_wait(BAR(C::B_VF + sv), (j / NSV) & 1, abort_flag, p.status, p.limit_ns)) break;
+        tc_fence_after();
+        const uint32_t p_tm = tmem + ((j & 1) ? C::TM_P1 : C::TM_P0);
 #pragma unroll
-          for (int k = 0; k < BS / 16; ++k) {
-            const uint64_t b = smem_desc_sw128(sV + s * C::KV_BYTES + k * 2048, C::BOX_KV, 1024);
-            mma_ts(tmem + C::TM_O, p_tm + k * 8, b, idesc_pv, (j > 0 || k > 0) ? 1u : 0u);
-          }
-          mma_commit(BAR(C::B_OD + (j & 1)));
-          mma_commit(BAR(C::B_KVE + s));
+        for (int k = 0; k < BS / 16; ++k) {
+          const uint64_t b = smem_desc_sw128(sV + sv * C::KV_BYTES + k * 2048, C::BOX_KV, 1024);
+          mma_ts(tmem + C::TM_O, p_tm + k * 8, b, idesc_pv, (j > 0 || k > 0) ? 1u : 0u);
         }
+        mma_commit(BAR(C::B_OD + (j & 1)));
+        mma_commit(BAR(C::B_VE + sv));
+        // S buffer (j & 1) is free again: start S_{j+2}
+        if (j + 2 < n && !issue_qk(j + 2)) break;
       }
       // every MMA issued so far must finish before TMEM is freed
       mma_commit(BAR(C::B_MMA));
@@ -245,7 +277,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     // ------------------------------------------------------------ softmax
     const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
     const int row = tid;                         // query row inside the tile
-    const int qpos = p.q_pos0 + qi * BS + row;
+    const int qpos = p.q_pos0 + qrow0 + row;
+    const int qpos_first = p.q_pos0 + qrow0;
+    const float c_l2 = p.scale_log2;             // logits in log2 units: s * c_l2
     float m_use = -INFINITY;                     // reference maximum, log2 units
     float l = 0.f;
     bool ok = true;
@@ -262,16 +296,20 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       tmem_wait_ld();
       const int len = s_len[j];
       const int kpos0 = s_pos[j];
-      float mx = -INFINITY;
+      // masking only for partial blocks and blocks that reach past the first query
+      const bool tok = p.mask == PBSA_MASK_TOKEN && kpos0 + BS - 1 > qpos_first;
+      if (len < BS || tok) {
 #pragma unroll
-      for (int c = 0; c < BS; ++c) {
-        float x = __uint_as_float(sr[c]) * p.scale_log2;
-        bool vis = c < len;
-        if (p.mask == PBSA_MASK_TOKEN) vis = vis && (kpos0 + c <= qpos);
-        x = vis ? x : -INFINITY;
-        sr[c] = __float_as_uint(x);
-        mx = fmaxf(mx, x);
+        for (int c = 0; c < BS; ++c) {
+          bool vis = c < len;
+          if (tok) vis = vis && (kpos0 + c <= qpos);
+          if (!vis) sr[c] = __float_as_uint(-INFINITY);
+        }
       }
+      float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+      for (int c = 0; c < BS; ++c) mx4[c & 3] = fmaxf(mx4[c & 3], __uint_as_float(sr[c]));
+      const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * c_l2;
       const float m_new = fmaxf(m_use, mx);
       float alpha = 1.f;
       bool rescale = false;
@@ -282,16 +320,16 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         m_use = m_new;
         rescale = true;
       }
-      const float m_ref = (m_use == -INFINITY) ? 0.f : m_use;
-      float rs = 0.f;
+      const float neg_m = (m_use == -INFINITY) ? 0.f : -m_use;
+      float rs4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int c = 0; c < BS; c += 2) {
-        const float p0 = ex2(__uint_as_float(sr[c]) - m_ref);
-        const float p1 = ex2(__uint_as_float(sr[c + 1]) - m_ref);
-        rs += p0 + p1;
+        const float p0 = ex2(fmaf(__uint_as_float(sr[c]), c_l2, neg_m));
+        const float p1 = ex2(fmaf(__uint_as_float(sr[c + 1]), c_l2, neg_m));
+        rs4[(c >> 1) & 3] += p0 + p1;
         sr[c >> 1] = pack_bf16x2(p0, p1);
       }
-      l = l * alpha + rs;
+      l = l * alpha + ((rs4[0] + rs4[1]) + (rs4[2] + rs4[3]));
       if (__any_sync(0xffffffffu, rescale)) {
         // O holds PV_0..PV_{j-1}: wait for the last of them, scale in place
         ok = mbar_wait(BAR(C::B_OD + ((j - 1) & 1)), ((j - 1) >> 1) & 1, abort_flag, p.status,
@@ -309,14 +347,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           tmem_st32(tmem + lane_base + C::TM_O + c * 32, orr);
         }
       }
-      if (j >= 2) {
-        // P buffer (j & 1) was last read by PV_{j-2}
-        ok = mbar_wait(BAR(C::B_OD + (j & 1)), ((j - 2) >> 1) & 1, abort_flag, p.status,
-                       p.limit_ns);
-        ok = __all_sync(0xffffffffu, ok);
-        if (!ok) break;
-        tc_fence_after();
-      }
+      // P buffer (j & 1) was last read by PV_{j-2}, which completed before S_j
+      // (issued after it) was signalled.
       const uint32_t p_tm = tmem + lane_base + ((j & 1) ? C::TM_P1 : C::TM_P0);
 #pragma unroll
       for (int c = 0; c < BS / 64; ++c)
@@ -335,7 +367,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       tc_fence_after();
       const bool valid = row < qlen;
       const float inv = l > 0.f ? 1.f / l : 0.f;
-      __nv_bfloat16* orow = p.o + (static_cast<long>(bh) * p.Tq + qi * BS + row) * D;
+      __nv_bfloat16* orow = p.o + (static_cast<long>(bh) * p.Tq + qrow0 + row) * D;
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t orr[32];
@@ -360,7 +392,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         }
       }
       if (valid)
-        p.lse[static_cast<long>(bh) * p.Tq + qi * BS + row] =
+        p.lse[static_cast<long>(bh) * p.Tq + qrow0 + row] =
             l > 0.f ? (m_use + __log2f(l)) * 0.69314718055994531f : -INFINITY;
     }
   }
@@ -373,19 +405,27 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   }
 }
 
-template <int D, int BS, int NST>
+template <int D, int BS, int NSK, int NSV>
 int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                const FwdParams& prm, cudaStream_t s) {
-  using C = FwdCfg<D, BS, NST>;
+  using C = FwdCfg<D, BS, NSK, NSV>;
   const size_t smem = C::smem_bytes(prm.Amax);
   PBSA_CHECK_ARG(smem <= 227 * 1024, PBSA_ERR_SHAPE, "attn_fwd: Amax too large for shared memory");
-  auto kern = attn_fwd_kernel<D, BS, NST>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(smem)) != cudaSuccess) {
-    PBSA_CHECK_LAUNCH("attn_fwd: cudaFuncSetAttribute");
+  auto kern = attn_fwd_kernel<D, BS, NSK, NSV>;
+  // opt in to the full 227 KB once per device (not a stream operation, so it
+  // also happens outside any graph capture after the first call)
+  static bool opted[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64 || !opted[dev]) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) !=
+        cudaSuccess) {
+      PBSA_CHECK_LAUNCH("attn_fwd: cudaFuncSetAttribute");
+    }
+    if (dev >= 0 && dev < 64) opted[dev] = true;
   }
   const long tiles = static_cast<long>(prm.B) * prm.H * prm.nQB;
-  kern<<<static_cast<unsigned>(tiles), 192, smem, s>>>(mq, mk, mv, prm);
+  kern<<<static_cast<unsigned>(tiles), kFwdThreads, smem, s>>>(mq, mk, mv, prm);
   PBSA_CHECK_LAUNCH("attn_fwd_kernel");
   return PBSA_OK;
 }
@@ -411,7 +451,7 @@ extern "C" int pbsa_attn_fwd(const pbsa_dims* d, const void* q, int Tq, int q_po
   PBSA_CHECK_ARG(aligned(q, 16) && aligned(kpool, 16) && aligned(vpool, 16) && aligned(o, 16),
                  PBSA_ERR_ALIGN, "attn_fwd: q, kpool, vpool and o must be 16-byte aligned");
   const long BH = static_cast<long>(d->B) * d->H;
-  const int nQB = (Tq + d->bs - 1) / d->bs;
+  const int nQB = qb_count(Tq, d->q_chunk, d->bs);
   PBSA_CHECK_ARG(BH * Tq < (1L << 31) && BH * NB * d->bs < (1L << 31), PBSA_ERR_SHAPE,
                  "attn_fwd: tensor rows must be < 2^31");
   PBSA_CHECK_ARG(BH * nQB < (1L << 31), PBSA_ERR_SHAPE, "attn_fwd: too many query tiles");
@@ -427,13 +467,13 @@ extern "C" int pbsa_attn_fwd(const pbsa_dims* d, const void* q, int Tq, int q_po
   FwdParams prm;
   prm.blk_len = blk_len; prm.blk_pos = blk_pos; prm.idx = idx; prm.cnt = cnt;
   prm.o = static_cast<__nv_bfloat16*>(o); prm.lse = lse;
-  prm.B = d->B; prm.H = d->H; prm.Tq = Tq; prm.q_pos0 = q_pos0; prm.NB = NB; prm.Amax = Amax;
+  prm.B = d->B; prm.H = d->H; prm.Tq = Tq; prm.q_chunk = d->q_chunk; prm.q_pos0 = q_pos0; prm.NB = NB; prm.Amax = Amax;
   prm.nQB = nQB; prm.mask = mask;
   prm.scale_log2 = d->scale * 1.4426950408889634f;
   prm.status = status; prm.limit_ns = wait_limit_ns(); prm.debug = debug_flags();
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (d->D == 128 && d->bs == 128) return launch_fwd<128, 128, 2>(mq, mk, mv, prm, s);
-  if (d->D == 64 && d->bs == 128) return launch_fwd<64, 128, 3>(mq, mk, mv, prm, s);
-  if (d->D == 128 && d->bs == 64) return launch_fwd<128, 64, 3>(mq, mk, mv, prm, s);
-  return launch_fwd<64, 64, 4>(mq, mk, mv, prm, s);
+  if (d->D == 128 && d->bs == 128) return launch_fwd<128, 128, 3, 2>(mq, mk, mv, prm, s);
+  if (d->D == 64 && d->bs == 128) return launch_fwd<64, 128, 4, 3>(mq, mk, mv, prm, s);
+  if (d->D == 128 && d->bs == 64) return launch_fwd<128, 64, 4, 3>(mq, mk, mv, prm, s);
+  return launch_fwd<64, 64, 4, 4>(mq, mk, mv, prm, s);
 }

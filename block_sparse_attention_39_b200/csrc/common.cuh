@@ -43,7 +43,27 @@ inline int common_dims_check(const pbsa_dims* d) {
   PBSA_CHECK_ARG(d->bs == 64 || d->bs == 128, PBSA_ERR_SHAPE, "bs must be 64 or 128");
   PBSA_CHECK_ARG(d->dtype == PBSA_BF16 || d->dtype == PBSA_FP32, PBSA_ERR_DTYPE,
                  "dtype must be PBSA_BF16 or PBSA_FP32");
+  PBSA_CHECK_ARG(d->q_chunk >= 0, PBSA_ERR_SHAPE, "q_chunk must be >= 0");
   return PBSA_OK;
+}
+
+// Query rows are chunks of qc rows (qc <= 0: one chunk), each tiled into
+// blocks of bs rows on its own.
+__host__ __device__ inline int qb_count(int Tq, int qc, int bs) {
+  qc = qc > 0 ? qc : Tq;
+  const int per = (qc + bs - 1) / bs;
+  const int full = Tq / qc;
+  const int rem = Tq - full * qc;
+  return full * per + (rem + bs - 1) / bs;
+}
+__host__ __device__ inline void qb_rows(int i, int Tq, int qc, int bs, int& row0, int& len) {
+  qc = qc > 0 ? qc : Tq;
+  const int per = (qc + bs - 1) / bs;
+  const int c = i / per, b = i - c * per;
+  const int crow = c * qc;
+  const int clen = min(qc, Tq - crow);
+  row0 = crow + b * bs;
+  len = min(bs, clen - b * bs);
 }
 
 inline size_t elem_size(int dtype) { return dtype == PBSA_BF16 ? 2 : 4; }

@@ -44,7 +44,7 @@ struct Vec16<float> {
 
 template <typename T, int D>
 __global__ void __launch_bounds__(kPoolThreads)
-pool_kernel(const T* __restrict__ q, int Tq, const T* __restrict__ kpool, int NB, int bs,
+pool_kernel(const T* __restrict__ q, int Tq, int qc, const T* __restrict__ kpool, int NB, int bs,
             const int32_t* __restrict__ blk_len, const int32_t* __restrict__ pool_ids, int nQB,
             float* __restrict__ q_bar, float* __restrict__ k_bar, int* status) {
   constexpr int EPC = Vec16<T>::EPC;
@@ -59,8 +59,9 @@ pool_kernel(const T* __restrict__ q, int Tq, const T* __restrict__ kpool, int NB
   float* out;
   int n;
   if (item < nQB) {
-    n = min(bs, Tq - item * bs);
-    base = q + (bh * Tq + static_cast<long>(item) * bs) * D;
+    int row0;
+    qb_rows(item, Tq, qc, bs, row0, n);
+    base = q + (bh * Tq + row0) * static_cast<long>(D);
     out = q_bar + (bh * nQB + item) * D;
   } else {
     const int id = pool_ids[item - nQB];
@@ -80,12 +81,23 @@ pool_kernel(const T* __restrict__ q, int Tq, const T* __restrict__ kpool, int NB
   float acc[EPC];
 #pragma unroll
   for (int e = 0; e < EPC; ++e) acc[e] = 0.f;
-  for (int r = rg; r < n; r += RPP) {
-    float x[EPC];
-    Vec16<T>::load(base + static_cast<long>(r) * D + c * EPC, x);
+  // a block has at most 128 rows: at most 128 / RPP loads per thread, all in flight together
+  constexpr int MAXR = (128 + RPP - 1) / RPP;
+  float x[MAXR][EPC];
 #pragma unroll
-    for (int e = 0; e < EPC; ++e) acc[e] += x[e];
+  for (int k = 0; k < MAXR; ++k) {
+    const int r = rg + k * RPP;
+    if (r < n) {
+      Vec16<T>::load(base + static_cast<long>(r) * D + c * EPC, x[k]);
+    } else {
+#pragma unroll
+      for (int e = 0; e < EPC; ++e) x[k][e] = 0.f;
+    }
   }
+#pragma unroll
+  for (int k = 0; k < MAXR; ++k)
+#pragma unroll
+    for (int e = 0; e < EPC; ++e) acc[e] += x[k][e];
   // lanes l and l ^ (CPR * 2^k) hold the same chunk
 #pragma unroll
   for (int off = CPR; off < 32; off <<= 1) {
@@ -114,21 +126,46 @@ __global__ void __launch_bounds__(256)
 score_kernel(const float* __restrict__ q_bar, const float* __restrict__ k_bar, int nQB, int NB,
              float scale, float* __restrict__ scores, float* __restrict__ mem) {
   __shared__ float kb[kScoreJ][D + 1];
-  __shared__ float qb[kScoreI][D];
+  __shared__ __align__(16) float qb[kScoreI][D];
   __shared__ float msum[8][kScoreJ];
   const long bh = blockIdx.y;
   const int j0 = blockIdx.x * kScoreJ;
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
-  for (int e = t; e < kScoreJ * D; e += 256) {
-    const int jj = e / D, d = e % D;
-    kb[jj][d] = (j0 + jj < NB) ? k_bar[(bh * NB + j0 + jj) * D + d] : 0.f;
+  {
+    // 32 x D floats as float4: (8 * D / 256) loads per thread, issued together
+    constexpr int NV = kScoreJ * D / 4 / 256;
+    float4 v[NV];
+#pragma unroll
+    for (int k = 0; k < NV; ++k) {
+      const int e = (t + k * 256) * 4;
+      const int jj = e / D;
+      v[k] = (j0 + jj < NB) ? *reinterpret_cast<const float4*>(k_bar + (bh * NB + j0 + jj) * D + e % D)
+                            : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int k = 0; k < NV; ++k) {
+      const int e = (t + k * 256) * 4;
+      float* dst = &kb[e / D][e % D];
+      dst[0] = v[k].x; dst[1] = v[k].y; dst[2] = v[k].z; dst[3] = v[k].w;
+    }
   }
   float macc = 0.f;
   const int j = j0 + lane;
   for (int i0 = 0; i0 < nQB; i0 += kScoreI) {
     const int ni = min(kScoreI, nQB - i0);
     __syncthreads();
-    for (int e = t; e < ni * D; e += 256) qb[e / D][e % D] = q_bar[(bh * nQB + i0) * D + e];
+    {
+      constexpr int NV = kScoreI * D / 4 / 256;
+      float4 v[NV];
+      const float4* src = reinterpret_cast<const float4*>(q_bar + (bh * nQB + i0) * D);
+#pragma unroll
+      for (int k = 0; k < NV; ++k) {
+        const int e4 = t + k * 256;
+        v[k] = (e4 * 4 < ni * D) ? src[e4] : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int k = 0; k < NV; ++k) reinterpret_cast<float4*>(&qb[0][0])[t + k * 256] = v[k];
+    }
     __syncthreads();
     for (int ii = warp; ii < ni; ii += 8) {
       float s = 0.f;
@@ -155,7 +192,7 @@ void launch_pool(const pbsa_dims* d, const void* q, int Tq, const void* kpool, i
                  float* q_bar, float* k_bar, int* status, cudaStream_t s) {
   dim3 grid(nQB + n_pool, d->B * d->H);
   pool_kernel<T, D><<<grid, kPoolThreads, 0, s>>>(
-      static_cast<const T*>(q), Tq, static_cast<const T*>(kpool), NB, d->bs, blk_len, pool_ids,
+      static_cast<const T*>(q), Tq, d->q_chunk, static_cast<const T*>(kpool), NB, d->bs, blk_len, pool_ids,
       nQB, q_bar, k_bar, status);
 }
 
@@ -179,7 +216,7 @@ extern "C" int pbsa_score_blocks(const pbsa_dims* d, const void* q, int Tq, cons
   PBSA_CHECK_ARG(aligned(q_bar, 4) && aligned(k_bar, 4) && aligned(scores, 4) &&
                      aligned(mem_score, 4) && aligned(blk_len, 4),
                  PBSA_ERR_ALIGN, "score_blocks: misaligned float/int buffer");
-  const int nQB = (Tq + d->bs - 1) / d->bs;
+  const int nQB = qb_count(Tq, d->q_chunk, d->bs);
   PBSA_CHECK_ARG(static_cast<long>(d->B) * d->H <= 65535, PBSA_ERR_SHAPE,
                  "score_blocks: B*H must be <= 65535");
   int* status = device_status_ptr();

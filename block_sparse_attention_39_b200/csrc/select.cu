@@ -24,35 +24,52 @@ __global__ void __launch_bounds__(32 * kSelWarps)
 select_kernel(const float* __restrict__ scores, int nQB, int NB, const int32_t* __restrict__ win_ids,
               int n_win, int k, const int32_t* __restrict__ mem_ids, int n_mem,
               const int32_t* __restrict__ blk_len, int mask, int q_pos0,
-              const int32_t* __restrict__ blk_pos, int Tq, int bs, int32_t* __restrict__ idx,
+              const int32_t* __restrict__ blk_pos, int Tq, int qc, int bs, int32_t* __restrict__ idx,
               int32_t* __restrict__ cnt, int Amax, int qb_offset, int nQB_total, int* status) {
   const int lane = threadIdx.x & 31;
   const int i = blockIdx.x * kSelWarps + (threadIdx.x >> 5);
   if (i >= nQB) return;
   const long bh = blockIdx.y;
   const float* srow = scores + (bh * nQB + i) * static_cast<long>(NB);
-  const int last_q = q_pos0 + i * bs + min(bs, Tq - i * bs) - 1;
+  int qrow0, qlen;
+  qb_rows(i, Tq, qc, bs, qrow0, qlen);
+  const int last_q = q_pos0 + qrow0 + qlen - 1;
 
-  // ---- Top-K over the window
+  // ---- gather: window ids and memory ids first, then their lengths/scores,
+  // so each lane has all of its loads in flight at once.  Memory entry e is
+  // held at element 255 - e (lane (255-e) / KPL, register (255-e) % KPL): the
+  // top `take` selected keys occupy elements [0, take) after the first sort
+  // and take + n_mem <= 256, so the two never collide.
+  int wid[KPL], mid[KPL];
+#pragma unroll
+  for (int r = 0; r < KPL; ++r) {
+    const int e = lane + 32 * r;               // coalesced over lanes
+    wid[r] = e < n_win ? win_ids[e] : -1;
+    const int me = 32 * KPL - 1 - (lane * KPL + r);
+    mid[r] = me < n_mem ? mem_ids[bh * n_mem + me] : -1;
+  }
+  int wlen[KPL], wpos[KPL], mlen[KPL];
+  float wsc[KPL];
+#pragma unroll
+  for (int r = 0; r < KPL; ++r) {
+    const int j = wid[r];
+    const bool in = j >= 0 && j < NB;
+    if (r * 32 + lane < n_win && !in) report_status(status, PBSA_ERR_ARG);
+    wlen[r] = in ? blk_len[bh * NB + j] : 0;
+    wsc[r] = in ? srow[j] : 0.f;
+    wpos[r] = (in && mask == PBSA_MASK_TOKEN) ? blk_pos[bh * NB + j] : 0;
+    const int m = mid[r];
+    mlen[r] = (m >= 0 && m < NB) ? blk_len[bh * NB + m] : 0;
+  }
+  // ---- Top-K over the window (element order is irrelevant before the sort)
   uint64_t key[KPL];
   int n_ok = 0;
 #pragma unroll
   for (int r = 0; r < KPL; ++r) {
-    const int e = lane * KPL + r;
-    key[r] = 0;
-    if (e < n_win) {
-      const int j = win_ids[e];
-      if (j < 0 || j >= NB) {
-        report_status(status, PBSA_ERR_ARG);
-        continue;
-      }
-      bool ok = blk_len[bh * NB + j] > 0;
-      if (ok && mask == PBSA_MASK_TOKEN) ok = blk_pos[bh * NB + j] <= last_q;
-      if (ok) {
-        key[r] = score_key(srow[j], static_cast<uint32_t>(j));
-        ++n_ok;
-      }
-    }
+    bool ok = wlen[r] > 0;
+    if (mask == PBSA_MASK_TOKEN) ok = ok && wpos[r] <= last_q;
+    key[r] = ok ? score_key(wsc[r], static_cast<uint32_t>(wid[r])) : 0ull;
+    n_ok += ok ? 1 : 0;
   }
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) n_ok += __shfl_xor_sync(0xffffffffu, n_ok, off);
@@ -66,9 +83,8 @@ select_kernel(const float* __restrict__ scores, int nQB, int NB, const int32_t* 
     uint64_t nk = 0;
     if (e < take) {
       nk = 0xffffffffull - key_id(key[r]);
-    } else if (e - take < n_mem) {
-      const int m = mem_ids[bh * n_mem + (e - take)];
-      if (m >= 0 && m < NB && blk_len[bh * NB + m] > 0) nk = 0xffffffffull - static_cast<uint32_t>(m);
+    } else if (mid[r] >= 0 && mid[r] < NB && mlen[r] > 0) {
+      nk = 0xffffffffull - static_cast<uint32_t>(mid[r]);
     }
     key[r] = nk;
   }
@@ -131,8 +147,8 @@ extern "C" int pbsa_select_local(const pbsa_dims* d, const float* scores, int nQ
                  "select_local: bad mask");
   PBSA_CHECK_ARG(mask == PBSA_MASK_CHUNK || blk_pos, PBSA_ERR_ARG,
                  "select_local: token mask needs blk_pos");
-  PBSA_CHECK_ARG(Tq >= 1 && (Tq + d->bs - 1) / d->bs == nQB, PBSA_ERR_SHAPE,
-                 "select_local: nQB must be ceil(Tq / bs)");
+  PBSA_CHECK_ARG(Tq >= 1 && qb_count(Tq, d->q_chunk, d->bs) == nQB, PBSA_ERR_SHAPE,
+                 "select_local: nQB must match the chunk tiling of Tq rows");
   PBSA_CHECK_ARG(qb_offset >= 0 && qb_offset + nQB <= nQB_total, PBSA_ERR_SHAPE,
                  "select_local: qb_offset + nQB must be <= nQB_total");
   PBSA_CHECK_ARG(static_cast<long>(d->B) * d->H <= 65535, PBSA_ERR_SHAPE,
@@ -142,7 +158,7 @@ extern "C" int pbsa_select_local(const pbsa_dims* d, const float* scores, int nQ
   dim3 grid((nQB + kSelWarps - 1) / kSelWarps, d->B * d->H);
   select_kernel<<<grid, 32 * kSelWarps, 0, static_cast<cudaStream_t>(stream)>>>(
       scores, nQB, NB, win_ids, n_win, k, mem_ids, n_mem, blk_len, mask, q_pos0, blk_pos, Tq,
-      d->bs, idx, cnt, Amax, qb_offset, nQB_total, status);
+      d->q_chunk, d->bs, idx, cnt, Amax, qb_offset, nQB_total, status);
   PBSA_CHECK_LAUNCH("select_kernel");
   return PBSA_OK;
 }

@@ -280,14 +280,23 @@ update_stash_kernel(UpdArgs a, const T* __restrict__ kpool, const T* __restrict_
   const long bh = blockIdx.y;
   PlanView pv = plan_view(a.ws, bh, a.P, a.M);
   if (!pv.stash[s]) return;
-  const long n16 = static_cast<long>(a.bs) * a.D * sizeof(T) / 16;
+  const int n16 = static_cast<int>(static_cast<long>(a.bs) * a.D * sizeof(T) / 16);
   const uint4* ks = reinterpret_cast<const uint4*>(kpool + (bh * a.NB + s) * static_cast<long>(a.bs) * a.D);
   const uint4* vs = reinterpret_cast<const uint4*>(vpool + (bh * a.NB + s) * static_cast<long>(a.bs) * a.D);
   uint4* kd = reinterpret_cast<uint4*>(stash + ((bh * a.P + s) * 2 + 0) * static_cast<long>(a.bs) * a.D);
   uint4* vd = reinterpret_cast<uint4*>(stash + ((bh * a.P + s) * 2 + 1) * static_cast<long>(a.bs) * a.D);
-  for (long e = threadIdx.x; e < n16; e += 256) {
-    kd[e] = ks[e];
-    vd[e] = vs[e];
+  for (int e0 = 0; e0 < n16; e0 += 256 * 8) {
+    uint4 ka[8], va[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const int e = e0 + threadIdx.x + k * 256;
+      if (e < n16) { ka[k] = ks[e]; va[k] = vs[e]; }
+    }
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const int e = e0 + threadIdx.x + k * 256;
+      if (e < n16) { kd[e] = ka[k]; vd[e] = va[k]; }
+    }
   }
 }
 
@@ -362,10 +371,27 @@ update_apply_kernel(UpdArgs a, T* __restrict__ kpool, T* __restrict__ vpool,
   const T* vb = vpool + (bh * a.NB + base) * blk_elems;
   if (m0 == m1) {
     // plain copy of a newly admitted block (base != s)
-    const long n16 = blk_elems * sizeof(T) / 16;
-    for (long e = t; e < n16; e += 256) {
-      reinterpret_cast<uint4*>(kd)[e] = reinterpret_cast<const uint4*>(kb)[e];
-      reinterpret_cast<uint4*>(vd)[e] = reinterpret_cast<const uint4*>(vb)[e];
+    // source and destination are different blocks of the same pool: load a
+    // batch of 16-byte chunks into registers, then store them
+    const int n16 = static_cast<int>(blk_elems * sizeof(T) / 16);
+    for (int e0 = 0; e0 < n16; e0 += 256 * 8) {
+      uint4 ka[8], va[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const int e = e0 + t + k * 256;
+        if (e < n16) {
+          ka[k] = reinterpret_cast<const uint4*>(kb)[e];
+          va[k] = reinterpret_cast<const uint4*>(vb)[e];
+        }
+      }
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const int e = e0 + t + k * 256;
+        if (e < n16) {
+          reinterpret_cast<uint4*>(kd)[e] = ka[k];
+          reinterpret_cast<uint4*>(vd)[e] = va[k];
+        }
+      }
     }
     if (t < D) kb_out[t] = a.k_bar[(bh * a.NB + base) * static_cast<long>(D) + t];
     if (t == 0) {

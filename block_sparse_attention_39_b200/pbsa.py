@@ -27,10 +27,12 @@ class PbsaError(RuntimeError):
         self.code = code
 
 
-def dims(B: int, H: int, D: int, bs: int, scale: float, dtype) -> PbsaDims:
+def dims(B: int, H: int, D: int, bs: int, scale: float, dtype, q_chunk: int = 0) -> PbsaDims:
+    """q_chunk: query rows per chunk, each chunk tiled into blocks on its own
+    (0: the whole query is one chunk)."""
     if isinstance(dtype, torch.dtype):
         dtype = BF16 if dtype == torch.bfloat16 else FP32
-    return PbsaDims(B, H, D, bs, float(scale), int(dtype))
+    return PbsaDims(B, H, D, bs, float(scale), int(dtype), int(q_chunk))
 
 
 def _p(t: Optional[torch.Tensor]):

@@ -23,7 +23,7 @@
  *      blk_len, blk_pos  [B, H, NB]   int32     (valid rows of a block; global
  *                                               token position of its row 0)
  *      k_bar             [B, H, NB, D] float    (pooled key of each block)
- *      q_bar             [B, H, nQB, D] float   nQB = ceil(Tq / bs)
+ *      q_bar             [B, H, nQB, D] float   nQB query blocks (see below)
  *      scores            [B, H, nQB, NB] float
  *      mem_score         [B, H, NB] float
  *      slot_src, slot_w  [B, H, P]    int32 / float  (persistent slots are
@@ -31,9 +31,13 @@
  *      idx               [B, H, nQB, Amax] int32 (attended physical ids,
  *                                               ascending, padded with -1)
  *      cnt               [B, H, nQB]  int32
- *  - Query block i covers rows [i*bs, min((i+1)*bs, Tq)); a chunk is tiled on
- *    its own, so its last block may be partial.  Rows of a block at or past
- *    blk_len are padding: never read as tokens.
+ *  - Query rows are a sequence of chunks of dims.q_chunk rows (the last chunk
+ *    may be shorter; q_chunk = 0 means one chunk of Tq rows).  Each chunk is
+ *    tiled into blocks of bs rows on its own, so the last block of every chunk
+ *    may be partial: with nb = ceil(q_chunk / bs), query block i covers rows
+ *    [c*q_chunk + b*bs, c*q_chunk + min((b+1)*bs, len_c)) for c = i / nb,
+ *    b = i % nb, len_c the rows of chunk c.  nQB counts these blocks.  Rows
+ *    of a cache block at or past blk_len are padding: never read as tokens.
  *  - Supported shapes: D in {64, 128}; bs in {64, 128}; B*H >= 1.
  *  - bf16 buffers must be 16-byte aligned (128-bit loads and TMA); float and
  *    int buffers 4-byte aligned.
@@ -72,11 +76,13 @@ typedef enum { PBSA_EVICT = 0, PBSA_MERGE_MEAN = 1 } pbsa_policy;
 typedef enum { PBSA_MASK_CHUNK = 0, PBSA_MASK_TOKEN = 1 } pbsa_mask;
 
 /* Problem dimensions shared by all calls.  scale multiplies <q, k> (usually
- * 1/sqrt(D)); dtype is the storage type of q, kpool and vpool. */
+ * 1/sqrt(D)); dtype is the storage type of q, kpool and vpool; q_chunk is the
+ * number of query rows per chunk (0: the whole query is one chunk). */
 typedef struct {
   int B, H, D, bs;
   float scale;
   int dtype; /* pbsa_dtype */
+  int q_chunk;
 } pbsa_dims;
 
 /* ---------------------------------------------------------------------------

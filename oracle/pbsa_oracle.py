@@ -74,26 +74,35 @@ def round_storage(x: np.ndarray, dtype: str) -> np.ndarray:
 # a1  block compression by pooling
 # ---------------------------------------------------------------------------
 
-def query_block_lengths(Tq: int, bs: int) -> np.ndarray:
-    """Query rows are tiled into ceil(Tq/bs) blocks, the last one partial (R9)."""
-    n = -(-Tq // bs)
-    lens = np.full(n, bs, dtype=np.int64)
-    if n:
-        lens[-1] = Tq - (n - 1) * bs
-    return lens
+def query_blocks(Tq: int, bs: int, q_chunk: int = 0):
+    """Query rows are a sequence of chunks of q_chunk rows (0: one chunk of Tq
+    rows; the last chunk may be shorter), and each chunk is tiled into blocks
+    of bs rows on its own, its last block partial (R9).  Returns the list of
+    (first row, length) of every query block."""
+    qc = q_chunk if q_chunk > 0 else Tq
+    out = []
+    for c0 in range(0, Tq, qc):
+        clen = min(qc, Tq - c0)
+        for b0 in range(0, clen, bs):
+            out.append((c0 + b0, min(bs, clen - b0)))
+    return out
 
 
-def pool_queries(q: np.ndarray, bs: int) -> np.ndarray:
+def query_block_lengths(Tq: int, bs: int, q_chunk: int = 0) -> np.ndarray:
+    return np.array([n for _, n in query_blocks(Tq, bs, q_chunk)], dtype=np.int64)
+
+
+def pool_queries(q: np.ndarray, bs: int, q_chunk: int = 0) -> np.ndarray:
     """Mean of the query rows of each query block (R1: mean over valid tokens).
 
     q: [B,H,Tq,D] -> q_bar [B,H,nQB,D] float64."""
     B, H, Tq, D = q.shape
-    lens = query_block_lengths(Tq, bs)
-    out = np.zeros((B, H, len(lens), D))
+    blocks = query_blocks(Tq, bs, q_chunk)
+    out = np.zeros((B, H, len(blocks), D))
     for b in range(B):
         for h in range(H):
-            for i, n in enumerate(lens):
-                rows = q[b, h, i * bs:i * bs + n].astype(np.float64)
+            for i, (r0, n) in enumerate(blocks):
+                rows = q[b, h, r0:r0 + n].astype(np.float64)
                 out[b, h, i] = rows.sum(axis=0) / n
     return out
 
@@ -137,9 +146,9 @@ def memory_scores(S: np.ndarray) -> np.ndarray:
     return S.sum(axis=2) / S.shape[2]
 
 
-def score_blocks(q, kpool, blk_len, pool_ids, k_bar, scale, bs):
+def score_blocks(q, kpool, blk_len, pool_ids, k_bar, scale, bs, q_chunk=0):
     """The whole scoring call: pool Q, (re)pool the listed key blocks, score all blocks."""
-    q_bar = pool_queries(q, bs)
+    q_bar = pool_queries(q, bs, q_chunk)
     k_bar = pool_keys(kpool, blk_len, pool_ids, k_bar)
     S = block_scores(q_bar, k_bar, scale)
     return q_bar, k_bar, S, memory_scores(S)
@@ -307,7 +316,8 @@ def update_memory(kpool, vpool, blk_len, blk_pos, k_bar, slot_src, slot_w,
 
 def select_local(S: np.ndarray, win_ids, k: int, mem_ids: Optional[np.ndarray],
                  blk_len: np.ndarray, mask: int = MASK_CHUNK, q_pos0: int = 0,
-                 blk_pos: Optional[np.ndarray] = None, bs: int = 0, Tq: int = 0):
+                 blk_pos: Optional[np.ndarray] = None, bs: int = 0, Tq: int = 0,
+                 q_chunk: int = 0):
     """Per query block: Top-K window blocks by block score, united with the memory.
 
     Inside the sliding window only the K most relevant blocks of each query
@@ -328,7 +338,7 @@ def select_local(S: np.ndarray, win_ids, k: int, mem_ids: Optional[np.ndarray],
     S: [B,H,nQB,NB] scores indexed by physical block id; mem_ids: [B,H,n_mem]
     physical ids (-1 = none) or None.  Returns a list of lists A[b][h][i]."""
     B, H, nQB, _ = S.shape
-    lens = query_block_lengths(Tq, bs) if mask == MASK_TOKEN else None
+    blocks = query_blocks(Tq, bs, q_chunk) if mask == MASK_TOKEN else None
     out = []
     for b in range(B):
         ob = []
@@ -344,7 +354,7 @@ def select_local(S: np.ndarray, win_ids, k: int, mem_ids: Optional[np.ndarray],
                     if blk_len[b, h, j] <= 0:
                         continue
                     if mask == MASK_TOKEN:
-                        last_q = q_pos0 + i * bs + int(lens[i]) - 1
+                        last_q = q_pos0 + blocks[i][0] + blocks[i][1] - 1
                         if blk_pos[b, h, j] > last_q:
                             continue
                     cands.append(j)
@@ -412,7 +422,7 @@ def _softmax_rows(s):
 
 
 def attention_fwd(q, kpool, vpool, blk_len, blk_pos, idx, cnt, scale: float,
-                  mask: int = MASK_CHUNK, q_pos0: int = 0):
+                  mask: int = MASK_CHUNK, q_pos0: int = 0, q_chunk: int = 0):
     """One softmax over the union of the attended blocks of each query block (R12).
 
     O_r = sum_c softmax_c(scale * <Q_r, K_c>) V_c over the valid tokens c of
@@ -423,13 +433,11 @@ def attention_fwd(q, kpool, vpool, blk_len, blk_pos, idx, cnt, scale: float,
     q: [B,H,Tq,D]; kpool/vpool [B,H,NB,bs,D]; idx [B,H,nQB,Amax]; cnt [B,H,nQB]."""
     B, H, Tq, D = q.shape
     bs = kpool.shape[3]
-    lens = query_block_lengths(Tq, bs)
     O = np.zeros((B, H, Tq, D))
     LSE = np.full((B, H, Tq), -np.inf)
     for b in range(B):
         for h in range(H):
-            for i, n in enumerate(lens):
-                r0 = i * bs
+            for i, (r0, n) in enumerate(query_blocks(Tq, bs, q_chunk)):
                 ids = [int(x) for x in idx[b, h, i, :cnt[b, h, i]]]
                 kc, vc, kpos = _gather_keys(kpool, vpool, blk_len, blk_pos, b, h, ids)
                 if kc.shape[0] == 0:
@@ -447,7 +455,7 @@ def attention_fwd(q, kpool, vpool, blk_len, blk_pos, idx, cnt, scale: float,
 # ---------------------------------------------------------------------------
 
 def attention_bwd(q, kpool, vpool, blk_len, blk_pos, idx, cnt, dO, scale: float,
-                  mask: int = MASK_CHUNK, q_pos0: int = 0):
+                  mask: int = MASK_CHUNK, q_pos0: int = 0, q_chunk: int = 0):
     """Gradients of ``attention_fwd`` w.r.t. Q, the key pool and the value pool.
 
     The attended lists are constants (R13: no gradient through selection).
@@ -457,14 +465,12 @@ def attention_bwd(q, kpool, vpool, blk_len, blk_pos, idx, cnt, dO, scale: float,
     to the block rows they were gathered from."""
     B, H, Tq, D = q.shape
     bs = kpool.shape[3]
-    lens = query_block_lengths(Tq, bs)
     dq = np.zeros((B, H, Tq, D))
     dk = np.zeros(kpool.shape)
     dv = np.zeros(vpool.shape)
     for b in range(B):
         for h in range(H):
-            for i, n in enumerate(lens):
-                r0 = i * bs
+            for i, (r0, n) in enumerate(query_blocks(Tq, bs, q_chunk)):
                 ids = [int(x) for x in idx[b, h, i, :cnt[b, h, i]]]
                 kc, vc, kpos = _gather_keys(kpool, vpool, blk_len, blk_pos, b, h, ids)
                 if kc.shape[0] == 0:

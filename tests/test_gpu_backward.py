@@ -1,0 +1,186 @@
+"""GPU parity of the attention backward (dQ, dK, dV) against the CPU oracle.
+
+The backward takes the forward's O (bf16) and LSE; here both come from the
+oracle (O rounded to bf16), so every input of the GPU call is independent of
+the CUDA path.  Gradients are compared with the oracle's exact float64
+gradients.  Tolerance: the attention bound plus one bf16 ulp (2^-8) of the
+gradient's own scale, because the tensor cores take P and dS rounded to bf16
+(relative error <= 2^-9 per term) and gradients, unlike O, are not bounded by
+the inputs' range:
+    max-abs  <= 2e-2 + 2^-8 * max|ref|,   mean-abs <= 2e-3 + 2^-8 * mean|ref|.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+import pbsa_inputs as PI
+from block_sparse_attention_39_b200 import pbsa as K
+from tests.gpu_util import dev_i32, dev_storage, host
+
+pytestmark = pytest.mark.gpu
+
+G_MAX, G_MEAN = 2e-2, 2e-3
+ULP = 2.0 ** -8
+
+
+def grad_ok(got, ref):
+    d = np.abs(got - ref)
+    mx, mean = float(d.max()), float(d.mean())
+    lim_mx = G_MAX + ULP * float(np.abs(ref).max())
+    lim_mean = G_MEAN + ULP * float(np.abs(ref).mean())
+    return mx <= lim_mx and mean <= lim_mean, (mx, lim_mx, mean, lim_mean)
+
+
+@pytest.fixture(autouse=True)
+def _status_clean():
+    assert torch.cuda.is_available()
+    K.get_status()
+    yield
+    assert K.get_status() == 0
+
+
+def _run_bwd(d, q, kp, vp, bl, bp, idx, cnt, q_pos0, mask, o, lse, dO):
+    B, H, Tq, D = q.shape
+    NB, bs = kp.shape[2], kp.shape[3]
+    Amax = idx.shape[-1]
+    ws = torch.empty(K.attn_bwd_workspace(d, Tq, NB, Amax), dtype=torch.uint8, device="cuda")
+    dq = torch.full((B, H, Tq, D), 3.0, dtype=torch.float32, device="cuda")
+    dk = torch.full((B, H, NB, bs, D), 3.0, dtype=torch.float32, device="cuda")
+    dv = torch.full((B, H, NB, bs, D), 3.0, dtype=torch.float32, device="cuda")
+    K.attn_bwd(d, dev_storage(q, "bf16"), Tq, q_pos0, dev_storage(kp, "bf16"),
+               dev_storage(vp, "bf16"), NB, dev_i32(bl), dev_i32(bp), dev_i32(idx), dev_i32(cnt),
+               Amax, mask, dev_storage(o, "bf16"), torch.from_numpy(lse.astype(np.float32)).cuda(),
+               dev_storage(dO, "bf16"), dq, dk, dv, ws)
+    torch.cuda.synchronize()
+    return host(dq), host(dk), host(dv)
+
+
+def _errs(got, ref, valid_rows_mask=None):
+    d = np.abs(got - ref)
+    return float(d.max()), float(d.mean())
+
+
+def _case(seed, B, H, D, bs, Tq, NB, Amax, mask, empty_rows=True):
+    r = np.random.default_rng(seed)
+    kp = O.round_bf16(r.standard_normal((B, H, NB, bs, D)))
+    vp = O.round_bf16(r.standard_normal((B, H, NB, bs, D)))
+    q = O.round_bf16(r.standard_normal((B, H, Tq, D)))
+    dO = O.round_bf16(r.standard_normal((B, H, Tq, D)))
+    bl = r.integers(1, bs + 1, size=(B, H, NB)).astype(np.int32)
+    bp = (np.arange(NB) * bs).astype(np.int32)[None, None, :].repeat(B, 0).repeat(H, 1)
+    nQB = -(-Tq // bs)
+    idx = np.full((B, H, nQB, Amax), -1, dtype=np.int32)
+    cnt = np.zeros((B, H, nQB), dtype=np.int32)
+    for b in range(B):
+        for h in range(H):
+            for i in range(nQB):
+                n = int(r.integers(0 if empty_rows else 1, Amax + 1))
+                idx[b, h, i, :n] = np.sort(r.choice(NB, size=n, replace=False))
+                cnt[b, h, i] = n
+    q_pos0 = int(bp[0, 0, -1])
+    return q, kp, vp, dO, bl, bp, idx, cnt, q_pos0
+
+
+@pytest.mark.parametrize("D,bs", [(128, 128), (64, 64), (128, 64), (64, 128)])
+@pytest.mark.parametrize("Tq", [50, 200, 384])
+@pytest.mark.parametrize("mask", [PI.MASK_CHUNK, PI.MASK_TOKEN])
+def test_backward_shapes_ragged_and_empty(D, bs, Tq, mask):
+    B, H, NB, Amax = 1, 3, 9, 6
+    q, kp, vp, dO, bl, bp, idx, cnt, q_pos0 = _case(D + bs + Tq + 31 * mask, B, H, D, bs, Tq, NB,
+                                                    Amax, mask)
+    scale = 1 / math.sqrt(D)
+    o, lse = O.attention_fwd(q, kp, vp, bl, bp, idx, cnt, scale, mask, q_pos0)
+    rq, rk, rv = O.attention_bwd(q, kp, vp, bl, bp, idx, cnt, dO, scale, mask, q_pos0)
+    d = K.dims(B, H, D, bs, scale, torch.bfloat16)
+    gq, gk, gv = _run_bwd(d, q, kp, vp, bl, bp, idx, cnt, q_pos0, mask, O.round_bf16(o), lse, dO)
+    for name, g, rf in (("dq", gq, rq), ("dk", gk, rk), ("dv", gv, rv)):
+        ok, info = grad_ok(g, rf)
+        assert ok, (name, info)
+
+
+@pytest.mark.parametrize("bs", [64, 128])
+@pytest.mark.parametrize("mask", [PI.MASK_CHUNK, PI.MASK_TOKEN])
+def test_backward_chunked_query_tiling(bs, mask):
+    # 500 query rows in chunks of 200: blocks tile each chunk on its own
+    B, H, D, NB, Amax, Tq, qc = 1, 2, 128, 9, 6, 500, 200
+    nQB = len(O.query_blocks(Tq, bs, qc))
+    q, kp, vp, dO, bl, bp, idx, cnt, q_pos0 = _case(bs + 7 * mask, B, H, D, bs, nQB * bs, NB, Amax,
+                                                    mask)
+    q, dO = q[:, :, :Tq], dO[:, :, :Tq]
+    scale = 1 / math.sqrt(D)
+    o, lse = O.attention_fwd(q, kp, vp, bl, bp, idx, cnt, scale, mask, q_pos0, q_chunk=qc)
+    rq, rk, rv = O.attention_bwd(q, kp, vp, bl, bp, idx, cnt, dO, scale, mask, q_pos0, q_chunk=qc)
+    d = K.dims(B, H, D, bs, scale, torch.bfloat16, q_chunk=qc)
+    gq, gk, gv = _run_bwd(d, q, kp, vp, bl, bp, idx, cnt, q_pos0, mask, O.round_bf16(o), lse, dO)
+    for name, g, rf in (("dq", gq, rq), ("dk", gk, rk), ("dv", gv, rv)):
+        ok, info = grad_ok(g, rf)
+        assert ok, (name, info)
+
+
+def _train_lists(w, q, kpool, blk_len):
+    """Oracle lists of the trainable path (one-shot selection per query chunk):
+    persistent = top-P blocks older than the window by the chunk's memory score,
+    local = top-k window blocks per query block by block score."""
+    kb = O.pool_keys(kpool, blk_len, range(w.NB_phys), np.zeros((w.B, w.H, w.NB_phys, w.D)))
+    nQB = w.n_chunks * w.nb_c
+    A = [[[None] * nQB for _ in range(w.H)] for _ in range(w.B)]
+    for t in range(w.n_chunks):
+        qt = q[:, :, t * w.chunk_tokens:(t + 1) * w.chunk_tokens]
+        S = O.block_scores(O.pool_queries(qt, w.bs), kb, w.scale)
+        m = O.memory_scores(S)
+        older = [p for c in range(0, max(0, t - w.W + 1)) for p in w.chunk_phys_ids(c)]
+        mem = O.select_local(m[:, :, None, :], older, w.P, None, blk_len)
+        mem_ids = np.full((w.B, w.H, w.P), -1, dtype=np.int32)
+        for b in range(w.B):
+            for h in range(w.H):
+                mem_ids[b, h, :len(mem[b][h][0])] = mem[b][h][0]
+        win = [p for c in w.window_chunks(t) for p in w.chunk_phys_ids(c)]
+        At = O.select_local(S, win, w.k, mem_ids, blk_len)
+        for b in range(w.B):
+            for h in range(w.H):
+                for i in range(w.nb_c):
+                    A[b][h][t * w.nb_c + i] = At[b][h][i]
+    return O.lists_to_arrays(A, w.P + w.k)
+
+
+@pytest.mark.slow
+def test_backward_train_shape_sampled_heads():
+    w = PI.WORKLOADS["train"]
+    chunks = [PI.chunk_tensors(w, t) for t in range(w.n_chunks)]
+    q = np.concatenate([c[0] for c in chunks], axis=2)
+    kpool = PI.pool_from_chunks(w, {t: c[1] for t, c in enumerate(chunks)})
+    vpool = PI.pool_from_chunks(w, {t: c[2] for t, c in enumerate(chunks)})
+    del chunks
+    blk_len, blk_pos = PI.chunk_layout(w, range(w.n_chunks))
+    T = q.shape[2]
+    dO = PI.grad_output(w, T)
+    idx, cnt = _train_lists(w, q, kpool, blk_len)
+    d = K.dims(w.B, w.H, w.D, w.bs, w.scale, torch.bfloat16, q_chunk=w.chunk_tokens)
+    # forward on the GPU with the oracle's lists (O, LSE feed the backward)
+    qd, kd, vd = dev_storage(q, "bf16"), dev_storage(kpool, "bf16"), dev_storage(vpool, "bf16")
+    o = torch.empty(w.B, w.H, T, w.D, dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty(w.B, w.H, T, dtype=torch.float32, device="cuda")
+    K.attn_fwd(d, qd, T, 0, kd, vd, w.NB_phys, dev_i32(blk_len), dev_i32(blk_pos), dev_i32(idx),
+               dev_i32(cnt), idx.shape[-1], w.mask, o, lse)
+    ws = torch.empty(K.attn_bwd_workspace(d, T, w.NB_phys, idx.shape[-1]), dtype=torch.uint8,
+                     device="cuda")
+    dq = torch.empty(w.B, w.H, T, w.D, dtype=torch.float32, device="cuda")
+    dk = torch.empty(w.B, w.H, w.NB_phys, w.bs, w.D, dtype=torch.float32, device="cuda")
+    dv = torch.empty_like(dk)
+    K.attn_bwd(d, qd, T, 0, kd, vd, w.NB_phys, dev_i32(blk_len), dev_i32(blk_pos), dev_i32(idx),
+               dev_i32(cnt), idx.shape[-1], w.mask, o, lse, dev_storage(dO, "bf16"), dq, dk, dv, ws)
+    torch.cuda.synchronize()
+    for (b, h) in [(0, 0), (1, 11)]:
+        sl = (slice(b, b + 1), slice(h, h + 1))
+        ro, rl = O.attention_fwd(q[sl], kpool[sl], vpool[sl], blk_len[sl], blk_pos[sl], idx[sl],
+                                 cnt[sl], w.scale, q_chunk=w.chunk_tokens)
+        mx, mean = _errs(host(o[sl]), ro)
+        assert mx <= 2e-2 and mean <= 2e-3, ("o", mx, mean)
+        rq, rk, rv = O.attention_bwd(q[sl], kpool[sl], vpool[sl], blk_len[sl], blk_pos[sl],
+                                     idx[sl], cnt[sl], dO[sl], w.scale, q_chunk=w.chunk_tokens)
+        for name, g, rf in (("dq", dq, rq), ("dk", dk, rk), ("dv", dv, rv)):
+            ok, info = grad_ok(host(g[sl]), rf)
+            assert ok, (name, b, h, info)

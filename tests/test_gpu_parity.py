@@ -231,6 +231,30 @@ def test_attention_shapes_ragged_and_empty(D, bs, Tq, mask):
     np.testing.assert_allclose(gl[fin], ref_l[fin], atol=2e-3, rtol=0)
 
 
+@pytest.mark.parametrize("bs", [64, 128])
+@pytest.mark.parametrize("mask", [PI.MASK_CHUNK, PI.MASK_TOKEN])
+def test_attention_chunked_query_tiling(bs, mask):
+    # 500 query rows in chunks of 200 (last chunk 100): blocks tile each chunk
+    B, H, D, NB, Amax, Tq, qc = 1, 2, 128, 9, 6, 500, 200
+    nQB = len(O.query_blocks(Tq, bs, qc))
+    q, kp, vp, bl, bp, idx, cnt, q_pos0 = _random_attention_case(bs + mask, B, H, D, bs, nQB * bs,
+                                                                 NB, Amax, mask)
+    q = q[:, :, :Tq]
+    scale = 1 / math.sqrt(D)
+    ref_o, ref_l = O.attention_fwd(q, kp, vp, bl, bp, idx, cnt, scale, mask, q_pos0, q_chunk=qc)
+    d = K.dims(B, H, D, bs, scale, torch.bfloat16, q_chunk=qc)
+    o = torch.zeros(B, H, Tq, D, dtype=torch.bfloat16, device="cuda")
+    lse = torch.zeros(B, H, Tq, dtype=torch.float32, device="cuda")
+    K.attn_fwd(d, dev_storage(q, "bf16"), Tq, q_pos0, dev_storage(kp, "bf16"),
+               dev_storage(vp, "bf16"), NB, dev_i32(bl), dev_i32(bp), dev_i32(idx), dev_i32(cnt),
+               Amax, mask, o, lse)
+    torch.cuda.synchronize()
+    mx, mean = attn_errors(host(o), ref_o)
+    assert mx <= ATT_MAX and mean <= ATT_MEAN, (mx, mean)
+    fin = np.isfinite(ref_l)
+    np.testing.assert_allclose(host(lse)[fin], ref_l[fin], atol=2e-3, rtol=0)
+
+
 def test_attention_long_lists_near_capacity():
     # 120 attended blocks per query block (longer than any workload's list)
     B, H, D, bs, Tq, NB, Amax = 1, 2, 128, 128, 256, 130, 120
