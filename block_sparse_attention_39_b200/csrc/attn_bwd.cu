@@ -27,6 +27,9 @@
 #include "tc_sm100.cuh"
 #include "tmap.h"
 
+#include <mutex>
+#include <string>
+
 namespace pbsa {
 namespace {
 
@@ -751,4 +754,79 @@ extern "C" int pbsa_attn_bwd(const pbsa_dims* d, const void* q, int Tq, int q_po
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (d->D == 128) return launch_bwd<128>(d, p, mq, mdo, mk, mv, workspace, L, s);
   return launch_bwd<64>(d, p, mq, mdo, mk, mv, workspace, L, s);
+}
+
+// ---------------------------------------------------------------------------
+// Backward without a caller-provided workspace.
+//
+// Some callers cannot hand this library a device buffer: a host process that
+// owns all device memory through its own pool and gives plugins no allocator
+// hook, or latency-critical code that must never enter the CUDA allocator
+// (cudaMalloc can synchronise the device and take milliseconds).  For them the
+// scratch of the backward (Delta, the attended-pair bitmap and the reverse
+// lists) lives in a fixed array of device memory that is part of the library
+// image: every GPU that loads libpbsa.so holds these 16 MiB until the process
+// exits.
+// ---------------------------------------------------------------------------
+namespace pbsa {
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = static_cast<size_t>(16) << 20;
+__device__ __align__(256) unsigned char g_bwd_scratch[kNoAllocScratchBytes];
+
+// Device address of g_bwd_scratch on the current device.  In host code the
+// array's name only stands in for the device symbol, so the address is looked
+// up once per device (with that device current) and cached.
+void* noalloc_scratch(std::string* err) {
+  static void* ptrs[64] = {nullptr};
+  static std::mutex mu;
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess || dev < 0 || dev >= 64) {
+    *err = std::string("cannot query the current device: ") + cudaGetErrorString(e);
+    return nullptr;
+  }
+  std::lock_guard<std::mutex> lock(mu);
+  if (ptrs[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_bwd_scratch);
+    if (e != cudaSuccess || p == nullptr) {
+      *err = std::string("cudaGetSymbolAddress of the backward scratch failed: ") +
+             cudaGetErrorString(e);
+      return nullptr;
+    }
+    ptrs[dev] = p;
+  }
+  return ptrs[dev];
+}
+
+}  // namespace
+}  // namespace pbsa
+
+extern "C" size_t pbsa_attn_bwd_noalloc_max_scratch(void) { return pbsa::kNoAllocScratchBytes; }
+
+extern "C" int pbsa_attn_bwd_noalloc(const pbsa_dims* d, const void* q, int Tq, int q_pos0,
+                                     const void* kpool, const void* vpool, int NB,
+                                     const int32_t* blk_len, const int32_t* blk_pos,
+                                     const int32_t* idx, const int32_t* cnt, int Amax, int mask,
+                                     const void* o, const float* lse, const void* dO, float* dq,
+                                     float* dk, float* dv, void* stream) {
+  using namespace pbsa;
+  int rc = common_dims_check(d);
+  if (rc) return rc;
+  PBSA_CHECK_ARG(Tq >= 1 && NB >= 1 && Amax >= 1, PBSA_ERR_SHAPE,
+                 "attn_bwd_noalloc: need Tq >= 1, NB >= 1, Amax >= 1");
+  const size_t need = pbsa_attn_bwd_workspace(d, Tq, NB, Amax);
+  PBSA_CHECK_ARG(need > 0 && need <= kNoAllocScratchBytes, PBSA_ERR_WORKSPACE,
+                 "attn_bwd_noalloc: this problem needs " + std::to_string(need) +
+                     " bytes of scratch, more than the built-in " +
+                     std::to_string(kNoAllocScratchBytes) +
+                     " bytes; use pbsa_attn_bwd with a workspace");
+  std::string err;
+  void* ws = noalloc_scratch(&err);
+  PBSA_CHECK_ARG(ws != nullptr, PBSA_ERR_CUDA, "attn_bwd_noalloc: " + err);
+  // The shared scratch keeps the previous call's contents; the backward clears
+  // the part that must start at zero (the pair bitmap) and fully rewrites the rest.
+  return pbsa_attn_bwd(d, q, Tq, q_pos0, kpool, vpool, NB, blk_len, blk_pos, idx, cnt, Amax, mask,
+                       o, lse, dO, dq, dk, dv, ws, kNoAllocScratchBytes, stream);
 }

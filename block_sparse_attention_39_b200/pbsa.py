@@ -104,6 +104,19 @@ def attn_bwd(d: PbsaDims, q, Tq, q_pos0, kpool, vpool, NB, blk_len, blk_pos, idx
         _p(workspace), workspace.numel() * workspace.element_size(), _s(stream)))
 
 
+def attn_bwd_noalloc(d: PbsaDims, q, Tq, q_pos0, kpool, vpool, NB, blk_len, blk_pos, idx, cnt, Amax,
+                     mask, o, lse, dO, dq, dk, dv, stream=None):
+    """The backward without a caller workspace: its scratch is a fixed device
+    array inside the library (see pbsa_attn_bwd_noalloc in include/pbsa.h)."""
+    _check("pbsa_attn_bwd_noalloc", lib().pbsa_attn_bwd_noalloc(
+        ctypes.byref(d), _p(q), Tq, q_pos0, _p(kpool), _p(vpool), NB, _p(blk_len), _p(blk_pos),
+        _p(idx), _p(cnt), Amax, mask, _p(o), _p(lse), _p(dO), _p(dq), _p(dk), _p(dv), _s(stream)))
+
+
+def attn_bwd_noalloc_max_scratch() -> int:
+    return int(lib().pbsa_attn_bwd_noalloc_max_scratch())
+
+
 def get_status(stream=None) -> int:
     """Synchronise the stream; return and clear the device status word."""
     return int(lib().pbsa_get_status(_s(stream)))

@@ -218,6 +218,41 @@ int pbsa_attn_bwd(const pbsa_dims* dims, const void* q, int Tq, int q_pos0,
                   void* workspace, size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * pbsa_attn_bwd_noalloc: the backward of pbsa_attn_fwd, as pbsa_attn_bwd, for
+ * callers that cannot give the library a device buffer.  The Sparse Forcing
+ * pages have no counterpart; this is an interface convenience.
+ *
+ * Who needs it: a host process that owns all device memory through its own
+ * pool and offers no allocator hook, or code that must never enter the CUDA
+ * allocator (cudaMalloc may synchronise the device and stall for
+ * milliseconds).  Arguments and results are those of pbsa_attn_bwd minus the
+ * workspace; the caller still passes every input and output buffer.
+ *
+ * Scratch: a fixed 16 MiB array of device memory inside the library (see
+ * pbsa_attn_bwd_noalloc_max_scratch).  Every GPU that loads the library keeps
+ * it allocated until the process exits.  Problems whose scratch
+ * (pbsa_attn_bwd_workspace) exceeds it are rejected with PBSA_ERR_WORKSPACE and
+ * nothing is launched.  The call allocates nothing: no cudaMalloc, no
+ * cudaFree, no allocating library routine.
+ *
+ * The first call on a device looks up the array's device address (once per
+ * device, with that device current); make that first call before any stream
+ * capture.  All calls share the one array, which keeps the previous call's
+ * contents (each call clears what must start at zero): calls that may overlap
+ * on the GPU -- different streams, or different host threads -- race on it
+ * and must be ordered by the caller.
+ * ------------------------------------------------------------------------- */
+int pbsa_attn_bwd_noalloc(const pbsa_dims* dims, const void* q, int Tq, int q_pos0,
+                          const void* kpool, const void* vpool, int NB,
+                          const int32_t* blk_len, const int32_t* blk_pos,
+                          const int32_t* idx, const int32_t* cnt, int Amax, int mask,
+                          const void* o, const float* lse, const void* dO,
+                          float* dq, float* dk, float* dv, void* stream);
+
+/* Size in bytes of the built-in scratch used by pbsa_attn_bwd_noalloc. */
+size_t pbsa_attn_bwd_noalloc_max_scratch(void);
+
+/* ---------------------------------------------------------------------------
  * Status and diagnostics (no counterpart on the pages).
  * ------------------------------------------------------------------------- */
 
