@@ -6,23 +6,24 @@
 // "Optimización").  Here both parts are one list of physical block ids per
 // query block, and one softmax runs over their union.
 //
-// Design (one CTA per 128-row query tile, 7 warps):
-//   warp 4      TMA producer of the Q tile and of K_j for every listed block j,
+// Design (one CTA per 128-row query tile, 11 warps):
+//   warp 8      TMA producer of the Q tile and of K_j for every listed block j,
 //               gathered by row coordinate from the block pool through an
 //               NSK-stage ring (128-byte swizzle); a K stage is released as
 //               soon as its QK^T has run; also allocates / frees TMEM;
-//   warp 6      TMA producer of V_j through an NSV-stage ring;
-//   warp 5      tcgen05 issuer (one thread): S_0, S_1 first; then for each j,
-//               O += P_j V_j (P_j read from TMEM) as soon as the softmax has
-//               written it, followed by S_{j+2} = Q K_{j+2}^T into the score
-//               buffer just freed -- so the tensor core runs PV_j and QK_{j+2}
-//               while the softmax warps handle block j+1;
-//   warps 0-3   softmax (thread = query row = TMEM lane): fp32 online softmax
-//               in the log2 domain with a lazily moved reference maximum
-//               (O in TMEM is rescaled only when the row maximum grows by
-//               more than 2^8), P packed to bf16 into TMEM, then the
-//               epilogue O / l and LSE.
-// TMEM (D = bs = 128): S0 | S1 | O | P0 | P1 = 128+128+128+64+64 columns.
+//   warp 10     TMA producer of V_j through an NSV-stage ring;
+//   warp 9      tcgen05 issuer (one thread): the blocks of the list are split
+//               into two streams (even and odd positions).  S_0, S_1 first; then
+//               for each j, O_{j&1} += P_j V_j as soon as stream j&1 has written
+//               P_j, followed by S_{j+2} = Q K_{j+2}^T into the same score
+//               buffer (MMAs issued by one thread run in order);
+//   warps 0-3   softmax of stream 0, warps 4-7 softmax of stream 1 (thread =
+//               query row = TMEM lane): fp32 online softmax in the log2 domain
+//               with a lazily moved reference maximum (O_h in TMEM is rescaled
+//               only when the row maximum grows by more than 2^8), P packed to
+//               bf16 over the stream's score buffer;
+//   epilogue    warps 0-3 merge the two streams' (m, l, O) and write O, LSE.
+// TMEM (D = bs = 128): S0 | S1 | O0 | O1 = 4 x 128 columns.
 // Every mbarrier wait is bounded; on time-out the CTA raises an abort flag,
 // records PBSA_ERR_TIMEOUT, drains its copies and MMAs, frees TMEM, returns.
 #include <cuda.h>
@@ -63,35 +64,37 @@ struct FwdCfg {
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + Q_BYTES;
   static constexpr int OFF_V = OFF_K + NSK * KV_BYTES;
-  static constexpr int OFF_BAR = OFF_V + NSV * KV_BYTES;
+  static constexpr int OFF_STAT = OFF_V + NSV * KV_BYTES;  // stream 1's m and l per row
+  static constexpr int OFF_BAR = OFF_STAT + 2 * 128 * 4;
   // barrier indices
   static constexpr int B_Q = 0;
   static constexpr int B_KF = 1;                         // + K stage
   static constexpr int B_KE = B_KF + NSK;                // + K stage
   static constexpr int B_VF = B_KE + NSK;                // + V stage
   static constexpr int B_VE = B_VF + NSV;                // + V stage
-  static constexpr int B_SF = B_VE + NSV;                // + S buffer (2)
-  static constexpr int B_PF = B_SF + 2;                  // + P buffer (2)
-  static constexpr int B_OD = B_PF + 2;                  // + parity of the PV (2)
-  static constexpr int B_MMA = B_OD + 2;
+  static constexpr int B_SF = B_VE + NSV;                // + stream (2)
+  static constexpr int B_PF = B_SF + 2;                  // + stream (2)
+  static constexpr int B_OD = B_PF + 2;                  // + stream (2)
+  static constexpr int B_ST = B_OD + 2;                  // stream 1's statistics written
+  static constexpr int B_MMA = B_ST + 1;
   static constexpr int NBAR = B_MMA + 1;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int OFF_IDS = OFF_MISC + 16;
-  // tensor-memory columns
+  // tensor-memory columns: per stream h a score buffer S_h (P_h written over
+  // its first BS/2 columns as packed bf16) and an output accumulator O_h
   static constexpr int TM_S0 = 0;
   static constexpr int TM_S1 = BS;
-  static constexpr int TM_O = 2 * BS;
-  static constexpr int TM_P0 = 2 * BS + D;
-  static constexpr int TM_P1 = TM_P0 + BS / 2;
-  static constexpr int TM_USED = TM_P1 + BS / 2;
+  static constexpr int TM_O0 = 2 * BS;
+  static constexpr int TM_O1 = 2 * BS + D;
+  static constexpr int TM_USED = 2 * BS + 2 * D;
   static constexpr int TM_COLS = TM_USED <= 256 ? 256 : 512;
   static_assert(TM_USED <= 512, "tensor memory budget");
   static size_t smem_bytes(int Amax) { return 1024 + OFF_IDS + 3 * 4 * static_cast<size_t>(Amax); }
 };
 
-// Warp roles: 0-3 softmax / epilogue, 4 K producer + TMEM owner, 5 MMA issuer,
-// 6 V producer.
-constexpr int kFwdThreads = 224;
+// Warp roles: 0-3 softmax stream 0 and epilogue, 4-7 softmax stream 1,
+// 8 K producer + TMEM owner, 9 MMA issuer, 10 V producer.
+constexpr int kFwdThreads = 352;
 
 template <int D, int BS, int NSK, int NSV>
 __global__ void __launch_bounds__(kFwdThreads, 1)
@@ -116,6 +119,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   const uint32_t sQ = smem_u32(smem + C::OFF_Q);
   const uint32_t sK = smem_u32(smem + C::OFF_K);
   const uint32_t sV = smem_u32(smem + C::OFF_V);
+  float* st_m1 = reinterpret_cast<float*>(smem + C::OFF_STAT);
+  float* st_l1 = st_m1 + 128;
   const uint32_t bar0 = smem_u32(smem + C::OFF_BAR);
   auto BAR = [&](int k) { return bar0 + 8u * static_cast<uint32_t>(k); };
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
@@ -134,11 +139,12 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       mbar_init(BAR(C::B_VF + s), 1);
       mbar_init(BAR(C::B_VE + s), 1);
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(BAR(C::B_SF + b), 1);
-      mbar_init(BAR(C::B_PF + b), 128);
-      mbar_init(BAR(C::B_OD + b), 1);
+    for (int h = 0; h < 2; ++h) {
+      mbar_init(BAR(C::B_SF + h), 1);
+      mbar_init(BAR(C::B_PF + h), 128);
+      mbar_init(BAR(C::B_OD + h), 1);
     }
+    mbar_init(BAR(C::B_ST), 128);
     mbar_init(BAR(C::B_MMA), 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -158,7 +164,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     s_len[e] = len;
     s_pos[e] = pos;
   }
-  if (warp == 4) {
+  if (warp == 8) {
     tmem_alloc(smem_u32(tmem_holder), C::TM_COLS);
     tmem_relinquish();
   }
@@ -167,7 +173,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
 
-  if (warp == 4) {
+  if (warp == 8) {
     // ------------------------------------------------------------ K producer
     if (lane == 0 && n > 0) {
       prefetch_tmap(&tmQ);
@@ -197,7 +203,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       }
     }
     __syncwarp();
-  } else if (warp == 6) {
+  } else if (warp == 10) {
     // ------------------------------------------------------------ V producer
     if (lane == 0 && n > 0) {
       prefetch_tmap(&tmV);
@@ -224,12 +230,12 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       }
     }
     __syncwarp();
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0 && n > 0) {
       constexpr uint32_t idesc_qk = idesc_bf16_f32(128, BS, false, false);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, false, true);
-      // S_j = Q K_j^T into S buffer (j & 1); frees K stage j % NSK when done
+      // S_j = Q K_j^T into the score buffer of stream j & 1; frees K stage j % NSK
       auto issue_qk = [&](int j) -> bool {
         const int s = j % NSK;
         if (!mbar_wait(BAR(C::B_KF + s), (j / NSK) & 1, abort_flag, p.status, p.limit_ns))
@@ -251,21 +257,23 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       bool ok = mbar_wait(BAR(C::B_Q), 0, abort_flag, p.status, p.limit_ns) && issue_qk(0) &&
                 (n < 2 || issue_qk(1));
       for (int j = 0; ok && j < n; ++j) {
-        // O += P_j V_j once the softmax has written P_j
-        if (!mbar_wait(BAR(C::B_PF + (j & 1)), (j >> 1) & 1, abort_flag, p.status, p.limit_ns))
-          break;
+        const int h = j & 1;
+        // O_h += P_j V_j once stream h has written P_j (over S_h)
+        if (!mbar_wait(BAR(C::B_PF + h), (j >> 1) & 1, abort_flag, p.status, p.limit_ns)) break;
         const int sv = j % NSV;
         if (!mbar_wait(BAR(C::B_VF + sv), (j / NSV) & 1, abort_flag, p.status, p.limit_ns)) break;
         tc_fence_after();
-        const uint32_t p_tm = tmem + ((j & 1) ? C::TM_P1 : C::TM_P0);
+        const uint32_t p_tm = tmem + (h ? C::TM_S1 : C::TM_S0);
+        const uint32_t o_tm = tmem + (h ? C::TM_O1 : C::TM_O0);
 #pragma unroll
         for (int k = 0; k < BS / 16; ++k) {
           const uint64_t b = smem_desc_sw128(sV + sv * C::KV_BYTES + k * 2048, C::BOX_KV, 1024);
-          mma_ts(tmem + C::TM_O, p_tm + k * 8, b, idesc_pv, (j > 0 || k > 0) ? 1u : 0u);
+          mma_ts(o_tm, p_tm + k * 8, b, idesc_pv, (j >= 2 || k > 0) ? 1u : 0u);
         }
-        mma_commit(BAR(C::B_OD + (j & 1)));
+        mma_commit(BAR(C::B_OD + h));
         mma_commit(BAR(C::B_VE + sv));
-        // S buffer (j & 1) is free again: start S_{j+2}
+        // S_{j+2} reuses S_h: tcgen05 MMAs from one thread run in issue order,
+        // so it is written only after PV_j has read P_j
         if (j + 2 < n && !issue_qk(j + 2)) break;
       }
       // every MMA issued so far must finish before TMEM is freed
@@ -275,24 +283,27 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     __syncwarp();
   } else {
     // ------------------------------------------------------------ softmax
-    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
-    const int row = tid;                         // query row inside the tile
+    const int h = warp >> 2;                     // stream: blocks j with j & 1 == h
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t S_tm = tmem + lane_base + (h ? C::TM_S1 : C::TM_S0);
+    const uint32_t O_tm = tmem + lane_base + (h ? C::TM_O1 : C::TM_O0);
+    const int row = tid & 127;                   // query row inside the tile
     const int qpos = p.q_pos0 + qrow0 + row;
     const int qpos_first = p.q_pos0 + qrow0;
     const float c_l2 = p.scale_log2;             // logits in log2 units: s * c_l2
     float m_use = -INFINITY;                     // reference maximum, log2 units
     float l = 0.f;
     bool ok = true;
-    for (int j = 0; j < n; ++j) {
-      ok = mbar_wait(BAR(C::B_SF + (j & 1)), (j >> 1) & 1, abort_flag, p.status, p.limit_ns);
+    int jj = 0;                                  // index of the block within the stream
+    for (int j = h; j < n; j += 2, ++jj) {
+      ok = mbar_wait(BAR(C::B_SF + h), jj & 1, abort_flag, p.status, p.limit_ns);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
-      const uint32_t s_tm = tmem + lane_base + ((j & 1) ? C::TM_S1 : C::TM_S0);
       uint32_t sr[BS];
 #pragma unroll
       for (int c = 0; c < BS / 32; ++c)
-        tmem_ld32(s_tm + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
+        tmem_ld32(S_tm + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
       tmem_wait_ld();
       const int len = s_len[j];
       const int kpos0 = s_pos[j];
@@ -313,7 +324,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       const float m_new = fmaxf(m_use, mx);
       float alpha = 1.f;
       bool rescale = false;
-      if (j == 0) {
+      if (jj == 0) {
         m_use = m_new;
       } else if (m_new > m_use + 8.f) {
         alpha = ex2(m_use - m_new);
@@ -331,75 +342,89 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       }
       l = l * alpha + ((rs4[0] + rs4[1]) + (rs4[2] + rs4[3]));
       if (__any_sync(0xffffffffu, rescale)) {
-        // O holds PV_0..PV_{j-1}: wait for the last of them, scale in place
-        ok = mbar_wait(BAR(C::B_OD + ((j - 1) & 1)), ((j - 1) >> 1) & 1, abort_flag, p.status,
-                       p.limit_ns);
-        ok = __all_sync(0xffffffffu, ok);
-        if (!ok) break;
-        tc_fence_after();
+        // O_h holds this stream's earlier blocks; their last PV (block j-2) was
+        // issued before S_j, whose completion was just observed.
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
           uint32_t orr[32];
-          tmem_ld32(tmem + lane_base + C::TM_O + c * 32, orr);
+          tmem_ld32(O_tm + c * 32, orr);
           tmem_wait_ld();
 #pragma unroll
           for (int e = 0; e < 32; ++e) orr[e] = __float_as_uint(__uint_as_float(orr[e]) * alpha);
-          tmem_st32(tmem + lane_base + C::TM_O + c * 32, orr);
+          tmem_st32(O_tm + c * 32, orr);
         }
       }
-      // P buffer (j & 1) was last read by PV_{j-2}, which completed before S_j
-      // (issued after it) was signalled.
-      const uint32_t p_tm = tmem + lane_base + ((j & 1) ? C::TM_P1 : C::TM_P0);
+      // P_j over the first BS/2 columns of S_h (its scores are in registers now)
 #pragma unroll
       for (int c = 0; c < BS / 64; ++c)
-        tmem_st32(p_tm + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
+        tmem_st32(S_tm + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(BAR(C::B_PF + (j & 1)));
+      mbar_arrive(BAR(C::B_PF + h));
     }
     // ------------------------------------------------------------ epilogue
-    if (ok && n > 0) {
-      ok = mbar_wait(BAR(C::B_OD + ((n - 1) & 1)), ((n - 1) >> 1) & 1, abort_flag, p.status,
-                     p.limit_ns);
+    const int n_h = (n - h + 1) / 2;             // blocks of this stream
+    if (ok && n_h > 0) {
+      ok = mbar_wait(BAR(C::B_OD + h), (n_h - 1) & 1, abort_flag, p.status, p.limit_ns);
       ok = __all_sync(0xffffffffu, ok);
     }
-    if (ok) {
-      tc_fence_after();
-      const bool valid = row < qlen;
-      const float inv = l > 0.f ? 1.f / l : 0.f;
-      __nv_bfloat16* orow = p.o + (static_cast<long>(bh) * p.Tq + qrow0 + row) * D;
+    if (h == 1) {
+      // hand this stream's statistics to stream 0, which writes the output
+      st_m1[row] = m_use;
+      st_l1[row] = l;
+      tc_fence_before();
+      mbar_arrive(BAR(C::B_ST));
+    } else {
+      bool ok1 = mbar_wait(BAR(C::B_ST), 0, abort_flag, p.status, p.limit_ns);
+      ok = __all_sync(0xffffffffu, ok && ok1);
+      if (ok) {
+        tc_fence_after();
+        const int n1 = n / 2;
+        const float m1 = st_m1[row], l1 = st_l1[row];
+        const float m = fmaxf(m_use, m1);
+        const float a0 = (m_use == -INFINITY) ? 0.f : ex2(m_use - m);
+        const float a1 = (m1 == -INFINITY || n1 == 0) ? 0.f : ex2(m1 - m);
+        const float lt = a0 * l + a1 * l1;
+        const float inv = lt > 0.f ? 1.f / lt : 0.f;
+        const float w0 = a0 * inv, w1 = a1 * inv;
+        const bool valid = row < qlen;
+        __nv_bfloat16* orow = p.o + (static_cast<long>(bh) * p.Tq + qrow0 + row) * D;
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t orr[32];
-        if (n > 0) {
-          tmem_ld32(tmem + lane_base + C::TM_O + c * 32, orr);
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o0[32], o1[32];
+          if (n > 0) tmem_ld32(tmem + lane_base + C::TM_O0 + c * 32, o0);
+          if (n1 > 0) tmem_ld32(tmem + lane_base + C::TM_O1 + c * 32, o1);
           tmem_wait_ld();
-        } else {
+          float v[32];
 #pragma unroll
-          for (int e = 0; e < 32; ++e) orr[e] = 0u;
-        }
-        if (valid) {
-          uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+          for (int e = 0; e < 32; ++e) {
+            float x = n > 0 ? __uint_as_float(o0[e]) * w0 : 0.f;
+            if (n1 > 0) x = fmaf(__uint_as_float(o1[e]), w1, x);
+            v[e] = x;
+          }
+          if (valid) {
+            uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
 #pragma unroll
-          for (int v = 0; v < 4; ++v) {
-            uint4 u;
-            u.x = pack_bf16x2(__uint_as_float(orr[8 * v + 0]) * inv, __uint_as_float(orr[8 * v + 1]) * inv);
-            u.y = pack_bf16x2(__uint_as_float(orr[8 * v + 2]) * inv, __uint_as_float(orr[8 * v + 3]) * inv);
-            u.z = pack_bf16x2(__uint_as_float(orr[8 * v + 4]) * inv, __uint_as_float(orr[8 * v + 5]) * inv);
-            u.w = pack_bf16x2(__uint_as_float(orr[8 * v + 6]) * inv, __uint_as_float(orr[8 * v + 7]) * inv);
-            dst[v] = u;
+            for (int q4 = 0; q4 < 4; ++q4) {
+              uint4 u;
+              u.x = pack_bf16x2(v[8 * q4 + 0], v[8 * q4 + 1]);
+              u.y = pack_bf16x2(v[8 * q4 + 2], v[8 * q4 + 3]);
+              u.z = pack_bf16x2(v[8 * q4 + 4], v[8 * q4 + 5]);
+              u.w = pack_bf16x2(v[8 * q4 + 6], v[8 * q4 + 7]);
+              dst[q4] = u;
+            }
           }
         }
+        if (valid)
+          p.lse[static_cast<long>(bh) * p.Tq + qrow0 + row] =
+              lt > 0.f ? (m + __log2f(lt)) * 0.69314718055994531f : -INFINITY;
       }
-      if (valid)
-        p.lse[static_cast<long>(bh) * p.Tq + qrow0 + row] =
-            l > 0.f ? (m_use + __log2f(l)) * 0.69314718055994531f : -INFINITY;
     }
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 4) {
+  if (warp == 8) {
     tc_fence_after();
     tmem_dealloc(tmem, C::TM_COLS);
   }
@@ -472,7 +497,11 @@ extern "C" int pbsa_attn_fwd(const pbsa_dims* d, const void* q, int Tq, int q_po
   prm.scale_log2 = d->scale * 1.4426950408889634f;
   prm.status = status; prm.limit_ns = wait_limit_ns(); prm.debug = debug_flags();
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (d->D == 128 && d->bs == 128) return launch_fwd<128, 128, 3, 2>(mq, mk, mv, prm, s);
+  if (d->D == 128 && d->bs == 128) {
+    if (FwdCfg<128, 128, 3, 3>::smem_bytes(Amax) <= 227 * 1024)
+      return launch_fwd<128, 128, 3, 3>(mq, mk, mv, prm, s);
+    return launch_fwd<128, 128, 3, 2>(mq, mk, mv, prm, s);
+  }
   if (d->D == 64 && d->bs == 128) return launch_fwd<64, 128, 4, 3>(mq, mk, mv, prm, s);
   if (d->D == 128 && d->bs == 64) return launch_fwd<128, 64, 4, 3>(mq, mk, mv, prm, s);
   return launch_fwd<64, 64, 4, 4>(mq, mk, mv, prm, s);
