@@ -388,7 +388,7 @@ def main():
                         "select_local": round(float(per[:, 2].mean()), 5),
                         "attn_fwd": round(ms_attn, 5)},
         "attended_gflop_per_step": round(flops / 1e9, 3),
-        "roofline": {"kernel": "attn_fwd_kernel<128,128,3,2>", "bound": "tensor",
+        "roofline": {"kernel": "attn_fwd_kernel (D=128, bs=128)", "bound": "tensor",
                      "achieved": round(attn_tflops, 2), "peak": peak, "unit": "TFLOP/s",
                      "frac": round(attn_tflops / peak, 4), "traffic": None,
                      "peak_kind": f"bf16_tflops burst, {pk_kind}"},

@@ -6,12 +6,12 @@
 // "Optimización").  Here both parts are one list of physical block ids per
 // query block, and one softmax runs over their union.
 //
-// Design (one CTA per 128-row query tile, 11 warps):
-//   warp 8      TMA producer of the Q tile and of K_j for every listed block j,
-//               gathered by row coordinate from the block pool through an
-//               NSK-stage ring (128-byte swizzle); a K stage is released as
-//               soon as its QK^T has run; also allocates / frees TMEM;
-//   warp 10     TMA producer of V_j through an NSV-stage ring;
+// Design (one CTA per 128-row query tile, 12 warps):
+//   warp 8      TMA producer of the Q tile and of K_j / V_j for every listed
+//               block j, gathered by row coordinate from the block pool through
+//               NSK- and NSV-stage rings (128-byte swizzle); a K stage is
+//               released as soon as its QK^T has run, a V stage after its PV;
+//               also allocates / frees TMEM;
 //   warp 9      tcgen05 issuer (one thread): the blocks of the list are split
 //               into two streams (even and odd positions).  S_0, S_1 first; then
 //               for each j, O_{j&1} += P_j V_j as soon as stream j&1 has written
@@ -33,6 +33,8 @@
 #include "common.cuh"
 #include "tc_sm100.cuh"
 #include "tmap.h"
+
+#include <string>
 
 namespace pbsa {
 namespace {
@@ -93,8 +95,18 @@ struct FwdCfg {
 };
 
 // Warp roles: 0-3 softmax stream 0 and epilogue, 4-7 softmax stream 1,
-// 8 K producer + TMEM owner, 9 MMA issuer, 10 V producer.
-constexpr int kFwdThreads = 352;
+// 8 TMA producer (Q, K and V) + TMEM owner, 9 MMA issuer, 10-11 idle.
+// Registers: launched with kFwdLaunchRegs per thread (384 x 168 = 64,512 of
+// the 65,536); the producer warpgroup (8-11) gives back down to kRegsLow and
+// the two softmax warpgroups take kRegsHigh: 8 x 32 x 224 + 4 x 32 x 56 =
+// 64,512, and per scheduler (warps w, w+4, w+8) 224 + 224 + 56 <= 512.  The
+// host refuses to launch unless the kernel was built with kFwdLaunchRegs.
+constexpr int kFwdThreads = 384;
+constexpr int kFwdLaunchRegs = 168;
+constexpr uint32_t kRegsLow = 56, kRegsHigh = 224;
+static_assert(kFwdThreads / 128 * 128 == kFwdThreads, "whole warpgroups");
+static_assert(8 * 32 * kRegsHigh + 4 * 32 * kRegsLow == kFwdThreads * kFwdLaunchRegs,
+              "register split must equal the launch allocation");
 
 template <int D, int BS, int NSK, int NSV>
 __global__ void __launch_bounds__(kFwdThreads, 1)
@@ -141,7 +153,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     }
     for (int h = 0; h < 2; ++h) {
       mbar_init(BAR(C::B_SF + h), 1);
-      mbar_init(BAR(C::B_PF + h), 128);
+      mbar_init(BAR(C::B_PF + h), 4);   // one arrival per softmax warp
       mbar_init(BAR(C::B_OD + h), 1);
     }
     mbar_init(BAR(C::B_ST), 128);
@@ -172,60 +184,54 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
-
+  if (warp >= 8) {
+  regs_dec<kRegsLow>();
   if (warp == 8) {
-    // ------------------------------------------------------------ K producer
+    // ------------------------------------------------------------ producer
+    // K_j and V_j in list order.  V_j waits for PV_{j-NSV}, which always
+    // completes before K_{j+1} is needed (QK_{j+1} is issued after PV_{j-1}).
     if (lane == 0 && n > 0) {
       prefetch_tmap(&tmQ);
       prefetch_tmap(&tmK);
+      prefetch_tmap(&tmV);
       const int q_row = bh * p.Tq + qrow0;
       mbar_expect_tx(BAR(C::B_Q), C::Q_BYTES);
 #pragma unroll
       for (int kb = 0; kb < C::KB; ++kb) tma_load_2d(sQ + kb * C::BOX_Q, &tmQ, BAR(C::B_Q), kb * 64, q_row);
-      int issued = 0;
+      const bool skip_v0 = (p.debug & 1) != 0;
+      int k_issued = 0, v_issued = 0;
       for (int j = 0; j < n; ++j) {
+        const int kv_row = (bh * p.NB + s_ids[j]) * BS;
         const int s = j % NSK;
         if (j >= NSK &&
             !mbar_wait(BAR(C::B_KE + s), ((j / NSK) & 1) ^ 1, abort_flag, p.status, p.limit_ns))
           break;
-        const int kv_row = (bh * p.NB + s_ids[j]) * BS;
         mbar_expect_tx(BAR(C::B_KF + s), C::KV_BYTES);
 #pragma unroll
         for (int kb = 0; kb < C::KB; ++kb)
           tma_load_2d(sK + s * C::KV_BYTES + kb * C::BOX_KV, &tmK, BAR(C::B_KF + s), kb * 64, kv_row);
-        issued = j + 1;
+        k_issued = j + 1;
+        const int sv = j % NSV;
+        if (j >= NSV &&
+            !mbar_wait(BAR(C::B_VE + sv), ((j / NSV) & 1) ^ 1, abort_flag, p.status, p.limit_ns))
+          break;
+        if (!(skip_v0 && j == 0)) {
+          mbar_expect_tx(BAR(C::B_VF + sv), C::KV_BYTES);
+#pragma unroll
+          for (int kb = 0; kb < C::KB; ++kb)
+            tma_load_2d(sV + sv * C::KV_BYTES + kb * C::BOX_KV, &tmV, BAR(C::B_VF + sv), kb * 64,
+                        kv_row);
+        }
+        v_issued = j + 1;
       }
       // no copy may still be in flight when the CTA leaves
       mbar_drain(BAR(C::B_Q), 0, p.status, p.limit_ns);
-      for (int s = 0; s < NSK && s < issued; ++s) {
-        const int jl = s + ((issued - 1 - s) / NSK) * NSK;   // last load issued to stage s
+      for (int s = 0; s < NSK && s < k_issued; ++s) {
+        const int jl = s + ((k_issued - 1 - s) / NSK) * NSK;   // last K load to stage s
         mbar_drain(BAR(C::B_KF + s), (jl / NSK) & 1, p.status, p.limit_ns);
       }
-    }
-    __syncwarp();
-  } else if (warp == 10) {
-    // ------------------------------------------------------------ V producer
-    if (lane == 0 && n > 0) {
-      prefetch_tmap(&tmV);
-      const bool skip_v0 = (p.debug & 1) != 0;
-      int issued = 0;
-      for (int j = 0; j < n; ++j) {
-        const int s = j % NSV;
-        if (j >= NSV &&
-            !mbar_wait(BAR(C::B_VE + s), ((j / NSV) & 1) ^ 1, abort_flag, p.status, p.limit_ns))
-          break;
-        if (!(skip_v0 && j == 0)) {
-          const int kv_row = (bh * p.NB + s_ids[j]) * BS;
-          mbar_expect_tx(BAR(C::B_VF + s), C::KV_BYTES);
-#pragma unroll
-          for (int kb = 0; kb < C::KB; ++kb)
-            tma_load_2d(sV + s * C::KV_BYTES + kb * C::BOX_KV, &tmV, BAR(C::B_VF + s), kb * 64,
-                        kv_row);
-        }
-        issued = j + 1;
-      }
-      for (int s = 0; s < NSV && s < issued; ++s) {
-        const int jl = s + ((issued - 1 - s) / NSV) * NSV;
+      for (int s = 0; s < NSV && s < v_issued; ++s) {
+        const int jl = s + ((v_issued - 1 - s) / NSV) * NSV;
         if (!(skip_v0 && jl == 0)) mbar_drain(BAR(C::B_VF + s), (jl / NSV) & 1, p.status, p.limit_ns);
       }
     }
@@ -258,10 +264,12 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                 (n < 2 || issue_qk(1));
       for (int j = 0; ok && j < n; ++j) {
         const int h = j & 1;
-        // O_h += P_j V_j once stream h has written P_j (over S_h)
-        if (!mbar_wait(BAR(C::B_PF + h), (j >> 1) & 1, abort_flag, p.status, p.limit_ns)) break;
+        // O_h += P_j V_j once stream h has written P_j (over S_h).  V_j is
+        // normally loaded long before, so it is checked first and PV_j goes
+        // out as soon as P_j lands.
         const int sv = j % NSV;
         if (!mbar_wait(BAR(C::B_VF + sv), (j / NSV) & 1, abort_flag, p.status, p.limit_ns)) break;
+        if (!mbar_wait(BAR(C::B_PF + h), (j >> 1) & 1, abort_flag, p.status, p.limit_ns)) break;
         tc_fence_after();
         const uint32_t p_tm = tmem + (h ? C::TM_S1 : C::TM_S0);
         const uint32_t o_tm = tmem + (h ? C::TM_O1 : C::TM_O0);
@@ -281,7 +289,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       mbar_drain(BAR(C::B_MMA), 0, p.status, p.limit_ns);
     }
     __syncwarp();
+  }
   } else {
+    regs_inc<kRegsHigh>();
     // ------------------------------------------------------------ softmax
     const int h = warp >> 2;                     // stream: blocks j with j & 1 == h
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
@@ -319,8 +329,12 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       }
       float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-      for (int c = 0; c < BS; ++c) mx4[c & 3] = fmaxf(mx4[c & 3], __uint_as_float(sr[c]));
-      const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * c_l2;
+      for (int c = 0; c < BS; c += 8) {
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          mx4[u] = max3(mx4[u], __uint_as_float(sr[c + 2 * u]), __uint_as_float(sr[c + 2 * u + 1]));
+      }
+      const float mx = max3(mx4[0], mx4[1], fmaxf(mx4[2], mx4[3])) * c_l2;
       const float m_new = fmaxf(m_use, mx);
       float alpha = 1.f;
       bool rescale = false;
@@ -332,15 +346,46 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         rescale = true;
       }
       const float neg_m = (m_use == -INFINITY) ? 0.f : -m_use;
-      float rs4[4] = {0.f, 0.f, 0.f, 0.f};
+      const uint64_t negm2 = f2(neg_m, neg_m);
+      const uint64_t cl2 = f2(c_l2, c_l2);
+      uint64_t rs2[2] = {0ull, 0ull};
+      if (len == BS && !tok) {
+        // no masked key: one pair in four takes the FMA-pipe exp2
 #pragma unroll
-      for (int c = 0; c < BS; c += 2) {
-        const float p0 = ex2(fmaf(__uint_as_float(sr[c]), c_l2, neg_m));
-        const float p1 = ex2(fmaf(__uint_as_float(sr[c + 1]), c_l2, neg_m));
-        rs4[(c >> 1) & 3] += p0 + p1;
-        sr[c >> 1] = pack_bf16x2(p0, p1);
+        for (int c = 0; c < BS; c += 2) {
+          const uint64_t x2 =
+              fma2(f2(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), cl2, negm2);
+          uint64_t p2;
+          if (((c >> 1) & 3) == 3) {
+            p2 = exp2_poly2(x2);
+          } else {
+            float x0, x1;
+            f2_split(x2, x0, x1);
+            p2 = f2(ex2(x0), ex2(x1));
+          }
+          rs2[(c >> 1) & 1] = add2(rs2[(c >> 1) & 1], p2);
+          float p0, p1;
+          f2_split(p2, p0, p1);
+          sr[c >> 1] = pack_bf16x2(p0, p1);
+        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < BS; c += 2) {
+          const uint64_t x2 =
+              fma2(f2(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), cl2, negm2);
+          float x0, x1;
+          f2_split(x2, x0, x1);
+          const uint64_t p2 = f2(ex2(x0), ex2(x1));
+          rs2[(c >> 1) & 1] = add2(rs2[(c >> 1) & 1], p2);
+          float p0, p1;
+          f2_split(p2, p0, p1);
+          sr[c >> 1] = pack_bf16x2(p0, p1);
+        }
       }
-      l = l * alpha + ((rs4[0] + rs4[1]) + (rs4[2] + rs4[3]));
+      float ra, rb, rc, rd;
+      f2_split(rs2[0], ra, rb);
+      f2_split(rs2[1], rc, rd);
+      l = l * alpha + ((ra + rb) + (rc + rd));
       if (__any_sync(0xffffffffu, rescale)) {
         // O_h holds this stream's earlier blocks; their last PV (block j-2) was
         // issued before S_j, whose completion was just observed.
@@ -360,7 +405,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         tmem_st32(S_tm + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(BAR(C::B_PF + h));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(BAR(C::B_PF + h));
     }
     // ------------------------------------------------------------ epilogue
     const int n_h = (n - h + 1) / 2;             // blocks of this stream
@@ -437,6 +483,22 @@ int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& 
   const size_t smem = C::smem_bytes(prm.Amax);
   PBSA_CHECK_ARG(smem <= 227 * 1024, PBSA_ERR_SHAPE, "attn_fwd: Amax too large for shared memory");
   auto kern = attn_fwd_kernel<D, BS, NSK, NSV>;
+  // the register split inside the kernel assumes this launch allocation
+  static int launch_regs[64] = {0};
+  int rdev = 0;
+  cudaGetDevice(&rdev);
+  if (rdev < 0 || rdev >= 64 || launch_regs[rdev] == 0) {
+    cudaFuncAttributes fa;
+    if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) PBSA_CHECK_LAUNCH("attn_fwd: attributes");
+    if (rdev >= 0 && rdev < 64) launch_regs[rdev] = fa.numRegs;
+    PBSA_CHECK_ARG(fa.numRegs == kFwdLaunchRegs, PBSA_ERR_CUDA,
+                   "attn_fwd: kernel built with " + std::to_string(fa.numRegs) +
+                       " registers per thread, the register split needs " +
+                       std::to_string(kFwdLaunchRegs));
+  } else {
+    PBSA_CHECK_ARG(launch_regs[rdev] == kFwdLaunchRegs, PBSA_ERR_CUDA,
+                   "attn_fwd: kernel register count does not match the register split");
+  }
   // opt in to the full 227 KB once per device (not a stream operation, so it
   // also happens outside any graph capture after the first call)
   static bool opted[64] = {false};

@@ -118,7 +118,7 @@ pool_kernel(const T* __restrict__ q, int Tq, int qc, const T* __restrict__ kpool
   }
 }
 
-constexpr int kScoreJ = 32;   // key blocks per CTA
+constexpr int kScoreJ = 32;   // key blocks per CTA (one per lane)
 constexpr int kScoreI = 32;   // query blocks staged per pass (static smem < 48 KB)
 
 template <int D>

@@ -17,9 +17,12 @@
 namespace pbsa {
 namespace {
 
-constexpr int KPL = 8;                  // keys per lane: 256 per warp
+constexpr int KPL = 8;                  // capacity: 256 keys per warp
 constexpr int kSelWarps = 4;
 
+// W: keys per lane of the window sort; U: keys per lane of the union sort
+// (32*W >= n_win, 32*U >= n_mem + min(k, n_win)); both <= KPL.
+template <int W, int U>
 __global__ void __launch_bounds__(32 * kSelWarps)
 select_kernel(const float* __restrict__ scores, int nQB, int NB, const int32_t* __restrict__ win_ids,
               int n_win, int k, const int32_t* __restrict__ mem_ids, int n_mem,
@@ -37,65 +40,81 @@ select_kernel(const float* __restrict__ scores, int nQB, int NB, const int32_t* 
 
   // ---- gather: window ids and memory ids first, then their lengths/scores,
   // so each lane has all of its loads in flight at once.  Memory entry e is
-  // held at element 255 - e (lane (255-e) / KPL, register (255-e) % KPL): the
-  // top `take` selected keys occupy elements [0, take) after the first sort
-  // and take + n_mem <= 256, so the two never collide.
-  int wid[KPL], mid[KPL];
+  // held at union element 32*U-1-e: the top `take` selected keys occupy
+  // elements [0, take) of the union and take + n_mem <= 32*U, so the two
+  // never collide.
+  int wid[W], mid[U];
 #pragma unroll
-  for (int r = 0; r < KPL; ++r) {
+  for (int r = 0; r < W; ++r) {
     const int e = lane + 32 * r;               // coalesced over lanes
     wid[r] = e < n_win ? win_ids[e] : -1;
-    const int me = 32 * KPL - 1 - (lane * KPL + r);
+  }
+#pragma unroll
+  for (int r = 0; r < U; ++r) {
+    const int me = 32 * U - 1 - (lane * U + r);
     mid[r] = me < n_mem ? mem_ids[bh * n_mem + me] : -1;
   }
-  int wlen[KPL], wpos[KPL], mlen[KPL];
-  float wsc[KPL];
+  int wlen[W], wpos[W], mlen[U];
+  float wsc[W];
 #pragma unroll
-  for (int r = 0; r < KPL; ++r) {
+  for (int r = 0; r < W; ++r) {
     const int j = wid[r];
     const bool in = j >= 0 && j < NB;
     if (r * 32 + lane < n_win && !in) report_status(status, PBSA_ERR_ARG);
     wlen[r] = in ? blk_len[bh * NB + j] : 0;
     wsc[r] = in ? srow[j] : 0.f;
     wpos[r] = (in && mask == PBSA_MASK_TOKEN) ? blk_pos[bh * NB + j] : 0;
+  }
+#pragma unroll
+  for (int r = 0; r < U; ++r) {
     const int m = mid[r];
     mlen[r] = (m >= 0 && m < NB) ? blk_len[bh * NB + m] : 0;
   }
   // ---- Top-K over the window (element order is irrelevant before the sort)
-  uint64_t key[KPL];
+  uint64_t wkey[W];
   int n_ok = 0;
 #pragma unroll
-  for (int r = 0; r < KPL; ++r) {
+  for (int r = 0; r < W; ++r) {
     bool ok = wlen[r] > 0;
     if (mask == PBSA_MASK_TOKEN) ok = ok && wpos[r] <= last_q;
-    key[r] = ok ? score_key(wsc[r], static_cast<uint32_t>(wid[r])) : 0ull;
+    wkey[r] = ok ? score_key(wsc[r], static_cast<uint32_t>(wid[r])) : 0ull;
     n_ok += ok ? 1 : 0;
   }
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) n_ok += __shfl_xor_sync(0xffffffffu, n_ok, off);
-  warp_bitonic_sort_desc<KPL>(key);
+  warp_bitonic_sort_desc<W>(wkey);
   const int take = min(k, n_ok);
 
-  // ---- union with the memory ids, ascending (descending sort of ~id)
+  // ---- union with the memory ids, ascending (descending sort of ~id).
+  // Sorted window element e (lane e / W, register e % W) moves to union
+  // element e (lane e / U, register e % U) through one shuffle per register.
+  uint64_t key[U];
 #pragma unroll
-  for (int r = 0; r < KPL; ++r) {
-    const int e = lane * KPL + r;
+  for (int r = 0; r < U; ++r) {
+    const int e = lane * U + r;                      // union element held here
+    const int src_lane = (e / W) & 31, src_reg = e % W;
+    uint64_t got = 0;
+#pragma unroll
+    for (int q = 0; q < W; ++q) {
+      const uint64_t v = __shfl_sync(0xffffffffu, wkey[q], src_lane);
+      if (q == src_reg) got = v;
+    }
     uint64_t nk = 0;
     if (e < take) {
-      nk = 0xffffffffull - key_id(key[r]);
+      nk = 0xffffffffull - key_id(got);
     } else if (mid[r] >= 0 && mid[r] < NB && mlen[r] > 0) {
       nk = 0xffffffffull - static_cast<uint32_t>(mid[r]);
     }
     key[r] = nk;
   }
-  warp_bitonic_sort_desc<KPL>(key);
+  warp_bitonic_sort_desc<U>(key);
 
   // ---- dedupe and write
-  uint64_t prev_last = __shfl_up_sync(0xffffffffu, key[KPL - 1], 1);
-  int keep[KPL];
+  uint64_t prev_last = __shfl_up_sync(0xffffffffu, key[U - 1], 1);
+  int keep[U];
   int mine = 0;
 #pragma unroll
-  for (int r = 0; r < KPL; ++r) {
+  for (int r = 0; r < U; ++r) {
     const uint64_t prev = (r == 0) ? ((lane == 0) ? ~0ull : prev_last) : key[r - 1];
     keep[r] = (key[r] != 0 && key[r] != prev) ? 1 : 0;
     mine += keep[r];
@@ -114,7 +133,7 @@ select_kernel(const float* __restrict__ scores, int nQB, int NB, const int32_t* 
     return;
   }
 #pragma unroll
-  for (int r = 0; r < KPL; ++r) {
+  for (int r = 0; r < U; ++r) {
     if (keep[r]) out[pos++] = static_cast<int32_t>(0xffffffffu - static_cast<uint32_t>(key[r]));
   }
   for (int e = total + lane; e < Amax; e += 32) out[e] = -1;
@@ -156,9 +175,17 @@ extern "C" int pbsa_select_local(const pbsa_dims* d, const float* scores, int nQ
   int* status = device_status_ptr();
   PBSA_CHECK_ARG(status != nullptr, PBSA_ERR_CUDA, "select_local: no device status word");
   dim3 grid((nQB + kSelWarps - 1) / kSelWarps, d->B * d->H);
-  select_kernel<<<grid, 32 * kSelWarps, 0, static_cast<cudaStream_t>(stream)>>>(
-      scores, nQB, NB, win_ids, n_win, k, mem_ids, n_mem, blk_len, mask, q_pos0, blk_pos, Tq,
-      d->q_chunk, d->bs, idx, cnt, Amax, qb_offset, nQB_total, status);
+  auto pick = [](int n) { return n <= 64 ? 2 : (n <= 128 ? 4 : 8); };
+  const int W = pick(n_win), U = pick(n_mem + take_max);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+#define PBSA_SEL(WW, UU)                                                                       \
+  if (W == WW && U == UU)                                                                      \
+    select_kernel<WW, UU><<<grid, 32 * kSelWarps, 0, st>>>(                                    \
+        scores, nQB, NB, win_ids, n_win, k, mem_ids, n_mem, blk_len, mask, q_pos0, blk_pos, Tq, \
+        d->q_chunk, d->bs, idx, cnt, Amax, qb_offset, nQB_total, status);
+  PBSA_SEL(2, 2) PBSA_SEL(2, 4) PBSA_SEL(2, 8) PBSA_SEL(4, 2) PBSA_SEL(4, 4) PBSA_SEL(4, 8)
+  PBSA_SEL(8, 2) PBSA_SEL(8, 4) PBSA_SEL(8, 8)
+#undef PBSA_SEL
   PBSA_CHECK_LAUNCH("select_kernel");
   return PBSA_OK;
 }

@@ -217,5 +217,70 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
+// --------------------------------------------------------- register split
+// Move registers between warpgroups (all 4 warps of a warpgroup execute it).
+template <uint32_t R>
+__device__ __forceinline__ void regs_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(R));
+}
+template <uint32_t R>
+__device__ __forceinline__ void regs_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(R));
+}
+
+// ------------------------------------------------------- packed fp32 pairs
+// sm_100 executes two fp32 operations per instruction on a 64-bit register pair.
+__device__ __forceinline__ uint64_t f2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_split(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// 2^x for a pair of x in [-126, 8], computed on the FMA pipe instead of the
+// special-function unit.  Method: split x = n + f with n = round(x) by adding
+// and subtracting 1.5 * 2^23 (the sum's low mantissa bits hold n), evaluate a
+// degree-3 polynomial for 2^f on [-1/2, 1/2] (coefficients fitted for this
+// library by weighted least squares on Chebyshev nodes, max relative error
+// 7.6e-5, far below the 2^-9 of the bf16 P it feeds), and add n to the
+// exponent field.  Inputs below -126 are clamped (their value is below 2^-126).
+__device__ __forceinline__ uint64_t exp2_poly2(uint64_t x) {
+  float x0, x1;
+  f2_split(x, x0, x1);
+  x0 = fmaxf(x0, -126.0f);
+  x1 = fmaxf(x1, -126.0f);
+  const uint64_t xc = f2(x0, x1);
+  const uint64_t magic = f2(12582912.0f, 12582912.0f);
+  const uint64_t t = add2(xc, magic);                                  // round to integer
+  const uint64_t nf = add2(t, f2(-12582912.0f, -12582912.0f));         // n as a float
+  const uint64_t fr = add2(xc, nf ^ 0x8000000080000000ull);           // f = x - n
+  uint64_t p = fma2(fr, f2(0.055186376f, 0.055186376f), f2(0.24261236f, 0.24261236f));
+  p = fma2(fr, p, f2(0.69325829f, 0.69325829f));
+  p = fma2(fr, p, f2(0.99992794f, 0.99992794f));
+  float p0, p1, t0, t1;
+  f2_split(p, p0, p1);
+  f2_split(t, t0, t1);
+  const float r0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
+  const float r1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
+  return f2(r0, r1);
+}
+
 }  // namespace tc
 }  // namespace pbsa

@@ -10,8 +10,8 @@
 // updates as part of the kernel's job.
 //
 // Three launches:
-//   plan   one CTA per (b,h): rank the candidates with a warp bitonic sort of
-//          64-bit keys, assign slots, choose merge targets by pooled-key dot
+//   plan   one CTA per (b,h): rank the candidates by their unique 64-bit keys
+//          (each thread counts the larger keys), assign slots, choose merge targets by pooled-key dot
 //          products, and write a per-slot plan into the workspace;
 //   stash  (merge policy only) copy the old content of every losing slot that
 //          is about to be overwritten and is still needed by a merge;
@@ -144,23 +144,16 @@ __global__ void __launch_bounds__(256) update_plan_kernel(UpdArgs a) {
   }
   __syncthreads();
 
-  // ---- rank: warp 0 sorts the 256 keys (8 per lane), descending
-  if (warp == 0) {
-    uint64_t k[8];
-#pragma unroll
-    for (int r = 0; r < 8; ++r) k[r] = skey[lane * 8 + r];
-    warp_bitonic_sort_desc<8>(k);
-    int nv = 0;
-#pragma unroll
-    for (int r = 0; r < 8; ++r) {
-      if (k[r] != 0) {
-        it_rank[static_cast<int>(k[r] & 0xff)] = lane * 8 + r;
-        ++nv;
-      }
-    }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) nv += __shfl_xor_sync(0xffffffffu, nv, off);
-    if (lane == 0) s_nvalid = nv;
+  // ---- rank: keys are unique (item index in the low bits), so an item's
+  // position in the descending order is the number of larger keys; all 256
+  // threads count at once.
+  {
+    const uint64_t mine = skey[t];
+    int rank = 0;
+    for (int u = 0; u < NI; ++u) rank += skey[u] > mine ? 1 : 0;
+    if (mine != 0) it_rank[t] = rank;
+    const int nv = __syncthreads_count(mine != 0 ? 1 : 0);
+    if (t == 0) s_nvalid = nv;
   }
   __syncthreads();
   const int n_valid = s_nvalid;
