@@ -31,7 +31,7 @@ SIGNATURES = {
                                    c_int, c_int, c_void_p, c_void_p, c_void_p, c_void_p, c_int,
                                    c_void_p, c_int, c_void_p, c_size_t, c_void_p]),
     "pbsa_select_local": (c_int, [P, c_void_p, c_int, c_int, c_void_p, c_int, c_int, c_void_p,
-                                  c_int, c_void_p, c_int, c_int, c_void_p, c_int, c_void_p,
+                                  c_int, c_int, c_void_p, c_int, c_int, c_void_p, c_int, c_void_p,
                                   c_void_p, c_int, c_int, c_int, c_void_p]),
     "pbsa_attn_fwd": (c_int, [P, c_void_p, c_int, c_int, c_void_p, c_void_p, c_int, c_void_p,
                               c_void_p, c_void_p, c_void_p, c_int, c_int, c_void_p, c_void_p,

@@ -8,8 +8,9 @@
 // Kernel 1 (pool): one CTA per block to pool (query blocks and the listed key
 // blocks), 128-bit loads, fp32 accumulation, warp-shuffle + shared-memory
 // reduction.  HBM-bound: every input byte is read once.
-// Kernel 2 (score): one CTA per (b,h, 32 key blocks); all query-block means
-// are staged in shared memory; writes S and the memory score.
+// Kernel 2 (score): one CTA per (b,h, 32 key blocks); the query-block means
+// are staged in shared memory; writes S and the memory score of every query
+// chunk (the mean of S over the chunk's query blocks).
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 
@@ -124,10 +125,10 @@ constexpr int kScoreI = 32;   // query blocks staged per pass (static smem < 48 
 template <int D>
 __global__ void __launch_bounds__(256)
 score_kernel(const float* __restrict__ q_bar, const float* __restrict__ k_bar, int nQB, int NB,
-             float scale, float* __restrict__ scores, float* __restrict__ mem) {
+             float scale, float* __restrict__ scores, float* __restrict__ mem, int per_group,
+             int groups) {
   __shared__ float kb[kScoreJ][D + 1];
   __shared__ __align__(16) float qb[kScoreI][D];
-  __shared__ float msum[8][kScoreJ];
   const long bh = blockIdx.y;
   const int j0 = blockIdx.x * kScoreJ;
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
@@ -149,7 +150,6 @@ score_kernel(const float* __restrict__ q_bar, const float* __restrict__ k_bar, i
       dst[0] = v[k].x; dst[1] = v[k].y; dst[2] = v[k].z; dst[3] = v[k].w;
     }
   }
-  float macc = 0.f;
   const int j = j0 + lane;
   for (int i0 = 0; i0 < nQB; i0 += kScoreI) {
     const int ni = min(kScoreI, nQB - i0);
@@ -171,18 +171,19 @@ score_kernel(const float* __restrict__ q_bar, const float* __restrict__ k_bar, i
       float s = 0.f;
 #pragma unroll 8
       for (int d = 0; d < D; ++d) s = fmaf(qb[ii][d], kb[lane][d], s);
-      s *= scale;
-      if (j < NB) scores[(bh * nQB + i0 + ii) * NB + j] = s;
-      macc += s;
+      if (j < NB) scores[(bh * nQB + i0 + ii) * NB + j] = s * scale;
     }
   }
-  msum[warp][lane] = macc;
+  // memory score: mean over the query blocks of each query chunk, summed in
+  // block order from the scores this CTA just wrote
   __syncthreads();
-  if (warp == 0 && j < NB) {
+  for (int e = t; e < groups * kScoreJ; e += 256) {
+    const int g = e / kScoreJ, jj = j0 + e % kScoreJ;
+    if (jj >= NB) continue;
+    const int i_lo = g * per_group, i_hi = min(nQB, (g + 1) * per_group);
     float m = 0.f;
-#pragma unroll
-    for (int w = 0; w < 8; ++w) m += msum[w][lane];
-    mem[bh * NB + j] = m / static_cast<float>(nQB);
+    for (int i = i_lo; i < i_hi; ++i) m += scores[(bh * nQB + i) * NB + jj];
+    mem[(bh * groups + g) * NB + jj] = m / static_cast<float>(i_hi - i_lo);
   }
 }
 
@@ -239,10 +240,15 @@ extern "C" int pbsa_score_blocks(const pbsa_dims* d, const void* q, int Tq, cons
   }
   PBSA_CHECK_LAUNCH("pool_kernel");
   dim3 grid((NB + kScoreJ - 1) / kScoreJ, d->B * d->H);
+  const int qc = d->q_chunk > 0 ? d->q_chunk : Tq;
+  const int per_group = (qc + d->bs - 1) / d->bs;
+  const int groups = (Tq + qc - 1) / qc;
   if (d->D == 128)
-    score_kernel<128><<<grid, 256, 0, s>>>(q_bar, k_bar, nQB, NB, d->scale, scores, mem_score);
+    score_kernel<128><<<grid, 256, 0, s>>>(q_bar, k_bar, nQB, NB, d->scale, scores, mem_score,
+                                           per_group, groups);
   else
-    score_kernel<64><<<grid, 256, 0, s>>>(q_bar, k_bar, nQB, NB, d->scale, scores, mem_score);
+    score_kernel<64><<<grid, 256, 0, s>>>(q_bar, k_bar, nQB, NB, d->scale, scores, mem_score,
+                                          per_group, groups);
   PBSA_CHECK_LAUNCH("score_kernel");
   return PBSA_OK;
 }

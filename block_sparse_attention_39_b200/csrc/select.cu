@@ -8,8 +8,8 @@
 //
 // One warp per (b, h, query block): the window's scores become 64-bit keys
 // (orderable score, ~id), a warp-wide bitonic sort over 256 keys held in
-// registers picks the Top-K, and a second bitonic sort merges the selection
-// with the memory ids into an ascending, duplicate-free list.
+// registers (up to 512 keys) picks the Top-K, and a second bitonic sort merges
+// the selection with the memory ids into an ascending, duplicate-free list.
 #include <cuda_runtime.h>
 
 #include "common.cuh"
@@ -17,7 +17,7 @@
 namespace pbsa {
 namespace {
 
-constexpr int KPL = 8;                  // capacity: 256 keys per warp
+constexpr int KPL = 16;                 // capacity: 512 keys per warp
 constexpr int kSelWarps = 4;
 
 // W: keys per lane of the window sort; U: keys per lane of the union sort
@@ -25,7 +25,7 @@ constexpr int kSelWarps = 4;
 template <int W, int U>
 __global__ void __launch_bounds__(32 * kSelWarps)
 select_kernel(const float* __restrict__ scores, int nQB, int NB, const int32_t* __restrict__ win_ids,
-              int n_win, int k, const int32_t* __restrict__ mem_ids, int n_mem,
+              int n_win, int k, const int32_t* __restrict__ mem_ids, int n_mem, int mem_ld,
               const int32_t* __restrict__ blk_len, int mask, int q_pos0,
               const int32_t* __restrict__ blk_pos, int Tq, int qc, int bs, int32_t* __restrict__ idx,
               int32_t* __restrict__ cnt, int Amax, int qb_offset, int nQB_total, int* status) {
@@ -33,7 +33,7 @@ select_kernel(const float* __restrict__ scores, int nQB, int NB, const int32_t* 
   const int i = blockIdx.x * kSelWarps + (threadIdx.x >> 5);
   if (i >= nQB) return;
   const long bh = blockIdx.y;
-  const float* srow = scores + (bh * nQB + i) * static_cast<long>(NB);
+  const float* srow = scores + (bh * nQB_total + qb_offset + i) * static_cast<long>(NB);
   int qrow0, qlen;
   qb_rows(i, Tq, qc, bs, qrow0, qlen);
   const int last_q = q_pos0 + qrow0 + qlen - 1;
@@ -52,7 +52,7 @@ select_kernel(const float* __restrict__ scores, int nQB, int NB, const int32_t* 
 #pragma unroll
   for (int r = 0; r < U; ++r) {
     const int me = 32 * U - 1 - (lane * U + r);
-    mid[r] = me < n_mem ? mem_ids[bh * n_mem + me] : -1;
+    mid[r] = me < n_mem ? mem_ids[bh * mem_ld + me] : -1;
   }
   int wlen[W], wpos[W], mlen[U];
   float wsc[W];
@@ -145,7 +145,7 @@ select_kernel(const float* __restrict__ scores, int nQB, int NB, const int32_t* 
 
 extern "C" int pbsa_select_local(const pbsa_dims* d, const float* scores, int nQB, int NB,
                                  const int32_t* win_ids, int n_win, int k, const int32_t* mem_ids,
-                                 int n_mem, const int32_t* blk_len, int mask, int q_pos0,
+                                 int n_mem, int mem_ld, const int32_t* blk_len, int mask, int q_pos0,
                                  const int32_t* blk_pos, int Tq, int32_t* idx, int32_t* cnt,
                                  int Amax, int qb_offset, int nQB_total, void* stream) {
   using namespace pbsa;
@@ -153,7 +153,7 @@ extern "C" int pbsa_select_local(const pbsa_dims* d, const float* scores, int nQ
   if (rc) return rc;
   PBSA_CHECK_ARG(scores && blk_len && idx && cnt, PBSA_ERR_ARG, "select_local: NULL buffer");
   PBSA_CHECK_ARG(n_win >= 0 && n_win <= 32 * KPL, PBSA_ERR_SHAPE,
-                 "select_local: n_win must be in [0, 256]");
+                 "select_local: n_win must be in [0, 512]");
   PBSA_CHECK_ARG(n_win == 0 || win_ids, PBSA_ERR_ARG, "select_local: win_ids is NULL");
   PBSA_CHECK_ARG(n_mem >= 0 && (n_mem == 0 || mem_ids), PBSA_ERR_ARG,
                  "select_local: mem_ids is NULL");
@@ -161,7 +161,10 @@ extern "C" int pbsa_select_local(const pbsa_dims* d, const float* scores, int nQ
                  "select_local: need k >= 0, nQB >= 1, NB >= 1, Amax >= 1");
   const int take_max = k < n_win ? k : n_win;
   PBSA_CHECK_ARG(n_mem + take_max <= Amax && n_mem + take_max <= 32 * KPL, PBSA_ERR_SHAPE,
-                 "select_local: n_mem + min(k, n_win) must be <= min(Amax, 256)");
+                 "select_local: n_mem + min(k, n_win) must be <= min(Amax, 512)");
+  PBSA_CHECK_ARG(mem_ld >= 0 && (mem_ld == 0 || mem_ld >= n_mem), PBSA_ERR_ARG,
+                 "select_local: mem_ld must be 0 or >= n_mem");
+  if (mem_ld == 0) mem_ld = n_mem;
   PBSA_CHECK_ARG(mask == PBSA_MASK_CHUNK || mask == PBSA_MASK_TOKEN, PBSA_ERR_ARG,
                  "select_local: bad mask");
   PBSA_CHECK_ARG(mask == PBSA_MASK_CHUNK || blk_pos, PBSA_ERR_ARG,
@@ -175,16 +178,18 @@ extern "C" int pbsa_select_local(const pbsa_dims* d, const float* scores, int nQ
   int* status = device_status_ptr();
   PBSA_CHECK_ARG(status != nullptr, PBSA_ERR_CUDA, "select_local: no device status word");
   dim3 grid((nQB + kSelWarps - 1) / kSelWarps, d->B * d->H);
-  auto pick = [](int n) { return n <= 64 ? 2 : (n <= 128 ? 4 : 8); };
+  auto pick = [](int n) { return n <= 64 ? 2 : (n <= 128 ? 4 : (n <= 256 ? 8 : 16)); };
   const int W = pick(n_win), U = pick(n_mem + take_max);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
 #define PBSA_SEL(WW, UU)                                                                       \
   if (W == WW && U == UU)                                                                      \
     select_kernel<WW, UU><<<grid, 32 * kSelWarps, 0, st>>>(                                    \
-        scores, nQB, NB, win_ids, n_win, k, mem_ids, n_mem, blk_len, mask, q_pos0, blk_pos, Tq, \
+        scores, nQB, NB, win_ids, n_win, k, mem_ids, n_mem, mem_ld, blk_len, mask, q_pos0,      \
+        blk_pos, Tq,                                                                           \
         d->q_chunk, d->bs, idx, cnt, Amax, qb_offset, nQB_total, status);
-  PBSA_SEL(2, 2) PBSA_SEL(2, 4) PBSA_SEL(2, 8) PBSA_SEL(4, 2) PBSA_SEL(4, 4) PBSA_SEL(4, 8)
-  PBSA_SEL(8, 2) PBSA_SEL(8, 4) PBSA_SEL(8, 8)
+  PBSA_SEL(2, 2) PBSA_SEL(2, 4) PBSA_SEL(2, 8) PBSA_SEL(2, 16) PBSA_SEL(4, 2) PBSA_SEL(4, 4)
+  PBSA_SEL(4, 8) PBSA_SEL(4, 16) PBSA_SEL(8, 2) PBSA_SEL(8, 4) PBSA_SEL(8, 8) PBSA_SEL(8, 16)
+  PBSA_SEL(16, 2) PBSA_SEL(16, 4) PBSA_SEL(16, 8) PBSA_SEL(16, 16)
 #undef PBSA_SEL
   PBSA_CHECK_LAUNCH("select_kernel");
   return PBSA_OK;

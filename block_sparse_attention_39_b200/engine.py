@@ -166,3 +166,105 @@ class PbsaLayer:
         self.update(ci, cs, stream=stream)
         self.select(t, stream=stream)
         self.attend(t, stream=stream)
+
+
+class PbsaTrain:
+    """Device state of the trainable path: a whole sequence of query chunks
+    attending its own block-tiled cache (no slots; the persistent set names
+    cache blocks in place), with forward and backward through the C ABI.
+
+    Lists are one-shot per query chunk t: the persistent set is the top-P
+    blocks older than the window by chunk t's memory score, the local set the
+    top-k window blocks per query block (``lists()``), or, for the density
+    sweep, the top ceil(d * allowed) of all allowed blocks per query block
+    (``lists(density=d)``)."""
+
+    def __init__(self, w: Workload, device="cuda"):
+        assert not w.slots_in_pool
+        self.w = w
+        dev = torch.device(device)
+        self.dev = dev
+        B, H, D, bs = w.B, w.H, w.D, w.bs
+        self.T = w.n_chunks * w.chunk_tokens
+        self.G = w.n_chunks
+        self.nQB = w.n_chunks * w.nb_c
+        self.NB = w.NB_phys
+        self.d = K.dims(B, H, D, bs, w.scale, torch.bfloat16, q_chunk=w.chunk_tokens)
+        self.d1 = K.dims(B, H, D, bs, w.scale, torch.bfloat16)
+        self.q = torch.zeros(B, H, self.T, D, dtype=torch.bfloat16, device=dev)
+        self.kpool = torch.zeros(B, H, self.NB, bs, D, dtype=torch.bfloat16, device=dev)
+        self.vpool = torch.zeros_like(self.kpool)
+        self.dO = torch.zeros(B, H, self.T, D, dtype=torch.bfloat16, device=dev)
+        self.blk_len = torch.zeros(B, H, self.NB, dtype=torch.int32, device=dev)
+        self.blk_pos = torch.zeros(B, H, self.NB, dtype=torch.int32, device=dev)
+        self.k_bar = torch.zeros(B, H, self.NB, D, dtype=torch.float32, device=dev)
+        self.q_bar = torch.zeros(B, H, self.nQB, D, dtype=torch.float32, device=dev)
+        self.scores = torch.zeros(B, H, self.nQB, self.NB, dtype=torch.float32, device=dev)
+        self.mem = torch.zeros(B, H, self.G, self.NB, dtype=torch.float32, device=dev)
+        self.mem_idx = torch.full((B, H, self.G, w.P), -1, dtype=torch.int32, device=dev)
+        self.mem_cnt = torch.zeros(B, H, self.G, dtype=torch.int32, device=dev)
+        self.Amax = self.NB                   # room for the dense (density 1) lists
+        self.idx = torch.full((B, H, self.nQB, self.Amax), -1, dtype=torch.int32, device=dev)
+        self.cnt = torch.zeros(B, H, self.nQB, dtype=torch.int32, device=dev)
+        self.o = torch.zeros(B, H, self.T, D, dtype=torch.bfloat16, device=dev)
+        self.lse = torch.zeros(B, H, self.T, dtype=torch.float32, device=dev)
+        self.dq = torch.zeros(B, H, self.T, D, dtype=torch.float32, device=dev)
+        self.dk = torch.zeros(B, H, self.NB, bs, D, dtype=torch.float32, device=dev)
+        self.dv = torch.zeros_like(self.dk)
+        self.ws = torch.empty(K.attn_bwd_workspace(self.d, self.T, self.NB, self.Amax),
+                              dtype=torch.uint8, device=dev)
+        self.all_ids = _i32(list(range(self.NB)), dev)
+        self._ids = {}
+
+    def ids(self, key, values):
+        t = self._ids.get(key)
+        if t is None:
+            t = _i32(list(values), self.dev)
+            self._ids[key] = t
+        return t
+
+    def set_meta(self):
+        w = self.w
+        lens = w.chunk_block_lens()
+        for t in range(w.n_chunks):
+            for j, pid in enumerate(w.chunk_phys_ids(t)):
+                self.blk_len[:, :, pid] = lens[j]
+                self.blk_pos[:, :, pid] = t * w.chunk_tokens + j * w.bs
+
+    def lists(self, density=None, stream=None):
+        w = self.w
+        K.score_blocks(self.d, self.q, self.T, self.kpool, self.NB, self.blk_len, self.all_ids,
+                       self.NB, self.q_bar, self.k_bar, self.scores, self.mem, stream)
+        for t in range(self.G):
+            if density is None:
+                older = [p for c in range(0, max(0, t - w.W + 1)) for p in w.chunk_phys_ids(c)]
+                if older:
+                    o_ids = self.ids(("older", t), older)
+                    K.select_local(self.d1, self.mem, 1, self.NB, o_ids, len(older), w.P, None, 0,
+                                   self.blk_len, 0, 0, None, w.bs, self.mem_idx, self.mem_cnt,
+                                   w.P, t, self.G, stream)
+                win = self.ids(("win", t), [p for c in w.window_chunks(t)
+                                            for p in w.chunk_phys_ids(c)])
+                K.select_local(self.d1, self.scores, w.nb_c, self.NB, win, win.numel(), w.k,
+                               self.mem_idx, w.P, self.blk_len, 0, t * w.chunk_tokens,
+                               self.blk_pos, w.chunk_tokens, self.idx, self.cnt, self.Amax,
+                               t * w.nb_c, self.nQB, stream, mem_ld=self.G * w.P,
+                               mem_offset=t * w.P)
+            else:
+                allowed = [p for c in range(t + 1) for p in w.chunk_phys_ids(c)]
+                kd = max(1, int(-(-density * len(allowed) // 1)))
+                a_ids = self.ids(("allowed", t), allowed)
+                K.select_local(self.d1, self.scores, w.nb_c, self.NB, a_ids, len(allowed), kd,
+                               None, 0, self.blk_len, 0, t * w.chunk_tokens, self.blk_pos,
+                               w.chunk_tokens, self.idx, self.cnt, self.Amax, t * w.nb_c,
+                               self.nQB, stream)
+
+    def fwd(self, stream=None):
+        K.attn_fwd(self.d, self.q, self.T, 0, self.kpool, self.vpool, self.NB, self.blk_len,
+                   self.blk_pos, self.idx, self.cnt, self.Amax, self.w.mask, self.o, self.lse,
+                   stream)
+
+    def bwd(self, stream=None):
+        K.attn_bwd(self.d, self.q, self.T, 0, self.kpool, self.vpool, self.NB, self.blk_len,
+                   self.blk_pos, self.idx, self.cnt, self.Amax, self.w.mask, self.o, self.lse,
+                   self.dO, self.dq, self.dk, self.dv, self.ws, stream)

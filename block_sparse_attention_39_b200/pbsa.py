@@ -78,9 +78,17 @@ def update_memory(d: PbsaDims, kpool, vpool, NB, blk_len, blk_pos, k_bar, P, n_s
 
 
 def select_local(d: PbsaDims, scores, nQB, NB, win_ids, n_win, k, mem_ids, n_mem, blk_len, mask,
-                 q_pos0, blk_pos, Tq, idx, cnt, Amax, qb_offset=0, nQB_total=None, stream=None):
+                 q_pos0, blk_pos, Tq, idx, cnt, Amax, qb_offset=0, nQB_total=None, stream=None,
+                 mem_ld=0, mem_offset=0):
+    """mem_ids may be a view into a larger int32 tensor: row (b,h) starts at
+    mem_offset + (b*H+h)*mem_ld elements of mem_ids' storage."""
+    mp = None
+    if mem_ids is not None:
+        if not mem_ids.is_cuda:
+            raise ValueError("PBSA tensors must live on a CUDA device")
+        mp = ctypes.c_void_p(mem_ids.data_ptr() + 4 * mem_offset)
     _check("pbsa_select_local", lib().pbsa_select_local(
-        ctypes.byref(d), _p(scores), nQB, NB, _p(win_ids), n_win, k, _p(mem_ids), n_mem,
+        ctypes.byref(d), _p(scores), nQB, NB, _p(win_ids), n_win, k, mp, n_mem, mem_ld,
         _p(blk_len), mask, q_pos0, _p(blk_pos), Tq, _p(idx), _p(cnt), Amax, qb_offset,
         nQB if nQB_total is None else nQB_total, _s(stream)))
 

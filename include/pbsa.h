@@ -25,7 +25,7 @@
  *      k_bar             [B, H, NB, D] float    (pooled key of each block)
  *      q_bar             [B, H, nQB, D] float   nQB query blocks (see below)
  *      scores            [B, H, nQB, NB] float
- *      mem_score         [B, H, NB] float
+ *      mem_score         [B, H, G, NB] float    G query chunks (1 if q_chunk = 0)
  *      slot_src, slot_w  [B, H, P]    int32 / float  (persistent slots are
  *                                               physical ids 0..P-1)
  *      idx               [B, H, nQB, Amax] int32 (attended physical ids,
@@ -96,7 +96,8 @@ typedef struct {
  *                      j in pool_ids only (other entries are left as they are;
  *                      a block of length 0 pools to zero)
  *   scores[b,h,i,j]  = scale * <q_bar[b,h,i], k_bar[b,h,j]>  for all j < NB
- *   mem_score[b,h,j] = mean over i of scores[b,h,i,j]
+ *   mem_score[b,h,g,j] = mean of scores[b,h,i,j] over the query blocks i of
+ *                      query chunk g (one chunk, g = 0, when dims.q_chunk = 0)
  *
  * q, kpool: dtype of dims (bf16 or fp32).  pool_ids: device int32 [n_pool],
  * the same list for every (b,h); n_pool may be 0.  Outputs are overwritten.
@@ -148,26 +149,27 @@ int pbsa_update_memory(const pbsa_dims* dims, void* kpool, void* vpool, int NB,
  * Local" (per-query Top-K of relevant blocks inside the sliding window) and
  * PBSA item "Atención Híbrida" (dense over the persistent memory).
  *
- * For each (b,h) and query block i < nQB of this call:
+ * For each (b,h) and query block i < nQB of this call (list row
+ * r = qb_offset + i of the nQB_total rows of scores, idx and cnt):
  *   candidates = win_ids[0..n_win) with blk_len > 0 (and, with PBSA_MASK_TOKEN,
  *                blk_pos <= q_pos0 + last row of block i);
- *   local      = the best min(k, #candidates) by scores[b,h,i,j] (descending;
+ *   local      = the best min(k, #candidates) by scores[b,h,r,j] (descending;
  *                ties: lower physical id first);
  *   list       = mem_ids[b,h,0..n_mem) entries >= 0 with blk_len > 0, united
  *                with local, ascending, without duplicates.
- * Written to idx[b,h,qb_offset+i,0..cnt) (rest -1) and cnt[b,h,qb_offset+i],
- * where idx/cnt have nQB_total query-block rows.
+ * Written to idx[b,h,r,0..cnt) (rest -1) and cnt[b,h,r].
  *
- * scores: [B,H,nQB,NB] float, indexed by the same physical ids as blk_len
- * and blk_pos [B,H,NB].  win_ids: device int32 [n_win], same for every
- * (b,h).  mem_ids: device int32 [B,H,n_mem] or NULL with n_mem = 0.
- * blk_pos may be NULL with PBSA_MASK_CHUNK.  Tq is this call's query rows
- * (used for the token mask).  Limits: n_win <= 256, n_mem + min(k, n_win) <=
- * min(Amax, 256).
+ * scores: [B,H,nQB_total,NB] float, indexed by the same physical ids as
+ * blk_len and blk_pos [B,H,NB].  win_ids: device int32 [n_win], same for every
+ * (b,h).  mem_ids: device int32, row (b,h) at mem_ids + (b*H+h)*mem_ld
+ * (mem_ld = 0 means n_mem), or NULL with n_mem = 0.  blk_pos may be NULL with
+ * PBSA_MASK_CHUNK.  Tq is this call's query rows (nQB must be their block
+ * count under dims.q_chunk; used for the token mask).
+ * Limits: n_win <= 512, n_mem + min(k, n_win) <= min(Amax, 512).
  * ------------------------------------------------------------------------- */
 int pbsa_select_local(const pbsa_dims* dims, const float* scores, int nQB, int NB,
                       const int32_t* win_ids, int n_win, int k,
-                      const int32_t* mem_ids, int n_mem,
+                      const int32_t* mem_ids, int n_mem, int mem_ld,
                       const int32_t* blk_len, int mask, int q_pos0, const int32_t* blk_pos,
                       int Tq, int32_t* idx, int32_t* cnt, int Amax,
                       int qb_offset, int nQB_total, void* stream);

@@ -64,7 +64,7 @@ def test_null_buffers_rejected():
                                  NULL, NULL, NULL) == -1
     assert lib.pbsa_attn_fwd(ctypes.byref(d), NULL, 10, 0, NULL, NULL, 4, NULL, NULL, NULL, NULL,
                              4, 0, NULL, NULL, NULL) == -1
-    assert lib.pbsa_select_local(ctypes.byref(d), NULL, 1, 4, NULL, 0, 1, NULL, 0, NULL, 0, 0,
+    assert lib.pbsa_select_local(ctypes.byref(d), NULL, 1, 4, NULL, 0, 1, NULL, 0, 0, NULL, 0, 0,
                                  NULL, 10, NULL, NULL, 4, 0, 1, NULL) == -1
 
 
@@ -100,8 +100,8 @@ def test_select_limits():
     d = _d()
     fake = ctypes.c_void_p(256)
     # n_mem + min(k, n_win) > Amax
-    assert lib.pbsa_select_local(ctypes.byref(d), fake, 1, 300, fake, 74, 16, fake, 24, fake, 0, 0,
-                                 NULL, 100, fake, fake, 39, 0, 1, NULL) == -2
+    assert lib.pbsa_select_local(ctypes.byref(d), fake, 1, 300, fake, 74, 16, fake, 24, 0, fake, 0,
+                                 0, NULL, 100, fake, fake, 39, 0, 1, NULL) == -2
     # window too long for one warp
-    assert lib.pbsa_select_local(ctypes.byref(d), fake, 1, 300, fake, 300, 16, NULL, 0, fake, 0, 0,
-                                 NULL, 100, fake, fake, 64, 0, 1, NULL) == -2
+    assert lib.pbsa_select_local(ctypes.byref(d), fake, 1, 600, fake, 600, 16, NULL, 0, 0, fake, 0,
+                                 0, NULL, 100, fake, fake, 64, 0, 1, NULL) == -2

@@ -18,7 +18,7 @@ import torch
 import oracle as O
 import pbsa_inputs as PI
 from block_sparse_attention_39_b200 import pbsa as K
-from tests.gpu_util import dev_i32, dev_storage, host
+from tests.gpu_util import band_ok, dev_i32, dev_storage, host
 
 pytestmark = pytest.mark.gpu
 
@@ -184,3 +184,57 @@ def test_backward_train_shape_sampled_heads():
         for name, g, rf in (("dq", dq, rq), ("dk", dk, rk), ("dv", dv, rv)):
             ok, info = grad_ok(host(g[sl]), rf)
             assert ok, (name, b, h, info)
+
+
+def _train_inputs(w):
+    chunks = [PI.chunk_tensors(w, t) for t in range(w.n_chunks)]
+    q = np.concatenate([c[0] for c in chunks], axis=2)
+    kpool = PI.pool_from_chunks(w, {t: c[1] for t, c in enumerate(chunks)})
+    vpool = PI.pool_from_chunks(w, {t: c[2] for t, c in enumerate(chunks)})
+    blk_len, blk_pos = PI.chunk_layout(w, range(w.n_chunks))
+    return q, kpool, vpool, blk_len, blk_pos
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("density", [None, 0.10, 1.0])
+def test_train_lists_built_on_gpu_match_oracle(density):
+    """The trainable path's lists, built by the library's own score/select calls
+    (one-shot per query chunk, or top fraction of allowed blocks), equal the
+    oracle's up to near-tie swaps."""
+    from block_sparse_attention_39_b200.engine import PbsaTrain
+    w = PI.variant(PI.WORKLOADS["train"], B=1, H=4)
+    q, kpool, vpool, blk_len, blk_pos = _train_inputs(w)
+    T = PbsaTrain(w)
+    T.q.copy_(dev_storage(q, "bf16"))
+    T.kpool.copy_(dev_storage(kpool, "bf16"))
+    T.vpool.copy_(dev_storage(vpool, "bf16"))
+    T.set_meta()
+    T.lists(density=density)
+    torch.cuda.synchronize()
+    idx, cnt = host(T.idx), host(T.cnt)
+    kb = O.pool_keys(kpool, blk_len, range(w.NB_phys), np.zeros((w.B, w.H, w.NB_phys, w.D)))
+    for t in range(w.n_chunks):
+        qt = q[:, :, t * w.chunk_tokens:(t + 1) * w.chunk_tokens]
+        S = O.block_scores(O.pool_queries(qt, w.bs), kb, w.scale)
+        m = O.memory_scores(S)
+        older = [p for c in range(0, max(0, t - w.W + 1)) for p in w.chunk_phys_ids(c)]
+        win = [p for c in w.window_chunks(t) for p in w.chunk_phys_ids(c)]
+        allowed = [p for c in range(t + 1) for p in w.chunk_phys_ids(c)]
+        for h in range(w.H):
+            for i in range(w.nb_c):
+                r = t * w.nb_c + i
+                lst = [int(x) for x in idx[0, h, r, :cnt[0, h, r]]]
+                assert lst == sorted(set(lst))
+                if density is None:
+                    mem = [x for x in lst if x in set(older)]
+                    loc = [x for x in lst if x in set(win)]
+                    assert len(mem) + len(loc) == len(lst)
+                    if older:
+                        ok, _ = band_ok(mem, {j: m[0, h, j] for j in older}, min(w.P, len(older)))
+                        assert ok, (t, h, i, "memory")
+                    ok, _ = band_ok(loc, {j: S[0, h, i, j] for j in win}, min(w.k, len(win)))
+                    assert ok, (t, h, i, "local")
+                else:
+                    kd = int(np.ceil(density * len(allowed)))
+                    ok, _ = band_ok(lst, {j: S[0, h, i, j] for j in allowed}, kd)
+                    assert ok, (t, h, i)
