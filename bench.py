@@ -50,6 +50,8 @@ def parse():
     ap.add_argument("--workload", default="decode", choices=["decode"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the trainable-path, dense-comparator and rollout measurements")
     return ap.parse_args()
 
 
@@ -276,6 +278,156 @@ class DecodeRunner:
         return ms, h2d, d2h
 
 
+# ----------------------------------------------------------------- extras
+def _timed(torch, fn, reps, flush=None):
+    """Mean device time (ms) of fn() over reps, L2 flushed before each."""
+    s = torch.cuda.current_stream()
+    ts = []
+    for _ in range(reps):
+        if flush is not None:
+            flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(s)
+        fn()
+        b.record(s)
+        ts.append((a, b))
+    torch.cuda.synchronize()
+    return float(np.mean([a.elapsed_time(b) for a, b in ts]))
+
+
+def _pair_flops(idx, cnt, blk_len, q_lens, D, per_pair):
+    total = 0
+    B, H, nQB = cnt.shape
+    for b in range(B):
+        for h in range(H):
+            for i in range(nQB):
+                ids = idx[b, h, i, :cnt[b, h, i]]
+                total += per_pair * int(q_lens[i]) * int(blk_len[b, h, ids].astype(np.int64).sum()) * D
+    return total
+
+
+def bench_train(torch, flush, reps=5):
+    """Trainable-path shape: forward and backward of the one-shot lists, and the
+    density sweep (the d = 1 lists are dense block-causal attention)."""
+    import pbsa_inputs as PI
+    from block_sparse_attention_39_b200.engine import PbsaTrain
+    w = PI.WORKLOADS["train"]
+    T = PbsaTrain(w)
+    g = torch.Generator(device="cuda").manual_seed(w.seed)
+    for t in (T.q, T.dO):
+        t.copy_(torch.randn(t.shape, generator=g, device="cuda").bfloat16())
+    for t in (T.kpool, T.vpool):
+        t.copy_(torch.randn(t.shape, generator=g, device="cuda").bfloat16())
+    T.set_meta()
+    lens = np.array([n for c in range(w.n_chunks) for n in w.chunk_block_lens()], dtype=np.int64)
+    bl = T.blk_len.cpu().numpy()
+    out = {"shape": f"B{w.B} H{w.H} D{w.D} bf16, {w.n_chunks} chunks x {w.chunk_tokens} tokens "
+                    f"= {T.T} tokens, {T.NB} blocks of {w.bs}, chunk-causal"}
+    runs = [("lists P32+k16", None)] + [(f"density {int(d * 100)}%", d) for d in PI.TRAIN_DENSITIES]
+    dense_fwd = dense_bwd = None
+    rows = {}
+    for name, dens in runs:
+        T.lists(density=dens)
+        torch.cuda.synchronize()
+        idx, cnt = T.idx.cpu().numpy(), T.cnt.cpu().numpy()
+        ffl = _pair_flops(idx, cnt, bl, lens, w.D, 4)
+        T.fwd()
+        ms_f = _timed(torch, T.fwd, reps, flush)
+        ms_b = _timed(torch, T.bwd, reps, flush)
+        rows[name] = {"attended_blocks_per_query_block": round(float(cnt.mean()), 2),
+                      "fwd_ms": round(ms_f, 4), "fwd_tflops": round(ffl / ms_f / 1e9, 1),
+                      "bwd_ms": round(ms_b, 4), "bwd_tflops": round(2.5 * ffl / ms_b / 1e9, 1)}
+        if dens == 1.0:
+            dense_fwd, dense_bwd = ms_f, ms_b
+    for name, r in rows.items():
+        r["fwd_speedup_vs_dense"] = round(dense_fwd / r["fwd_ms"], 2)
+        r["bwd_speedup_vs_dense"] = round(dense_bwd / r["bwd_ms"], 2)
+    out["runs"] = rows
+    out["flop_count"] = "fwd 4*len_q*len_k*D, bwd 10*len_q*len_k*D per attended block pair"
+    del T
+    torch.cuda.empty_cache()
+    return out
+
+
+def bench_dense_comparators(torch, runner, flush, reps=10):
+    """The decode inputs through the same attention kernel with full lists:
+    the whole cache (185 blocks) and the sliding window alone (last 2 chunks)."""
+    from block_sparse_attention_39_b200 import pbsa as K
+    L, w = runner.L, runner.w
+    out = {}
+    for name, chunks in (("dense_full_cache", list(range(w.n_chunks))),
+                         ("dense_sliding_window", w.window_chunks(w.n_chunks - 1))):
+        ids = [p for c in chunks for p in w.chunk_phys_ids(c)]
+        idx = torch.tensor(ids, dtype=torch.int32, device="cuda").expand(
+            w.B, w.H, L.nQB, len(ids)).contiguous()
+        cnt = torch.full((w.B, w.H, L.nQB), len(ids), dtype=torch.int32, device="cuda")
+        fn = lambda: K.attn_fwd(L.dbf, L.q, w.chunk_tokens, runner.t * w.chunk_tokens, L.kpool,
+                                L.vpool, L.NB, L.blk_len, L.blk_pos, idx, cnt, len(ids), w.mask,
+                                L.o, L.lse)
+        fn()
+        ms = _timed(torch, fn, reps, flush)
+        lens = np.array(w.chunk_block_lens(), dtype=np.int64)
+        fl = 4 * int(lens.sum()) * int(np.array([w.chunk_block_lens()[i % w.nb_c] for i in range(len(ids))]).sum()) * w.D * w.B * w.H
+        out[name] = {"blocks": len(ids), "ms": round(ms, 4), "tflops": round(fl / ms / 1e9, 1)}
+    return out
+
+
+def layer_bytes(L):
+    """Library-owned device bytes of one layer's PBSA state (pool, metadata,
+    pooled keys, slots, workspace)."""
+    ts = [L.kpool, L.vpool, L.blk_len, L.blk_pos, L.k_bar, L.slot_src, L.slot_w, L.ws]
+    return int(sum(t.numel() * t.element_size() for t in ts))
+
+
+def bench_rollouts(torch, timed_steps=6):
+    """Per-chunk latency of the rollout workloads (score -> update -> select ->
+    attend per layer) on device-drawn N(0,1) inputs, and their KV bytes."""
+    import pbsa_inputs as PI
+    from block_sparse_attention_39_b200.engine import PbsaLayer
+    out = {}
+    g = torch.Generator(device="cuda").manual_seed(7)
+    for name in ("rollout20s", "rollout1min"):
+        w = PI.WORKLOADS[name]
+        layers = [PbsaLayer(w) for _ in range(w.layers)]
+        shape = (w.B, w.H, w.chunk_tokens, w.D)
+        warm = 4
+        steps = warm + timed_steps
+        def draw():
+            return tuple(torch.randn(shape, generator=g, device="cuda").bfloat16() for _ in range(3))
+        times = []
+        for t in range(steps):
+            if t >= warm:
+                pre = [draw() for _ in layers]          # drawn before the timed region
+            s = torch.cuda.current_stream()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            for li, L in enumerate(layers):
+                q, k, v = pre[li] if t >= warm else draw()
+                L.write_chunk(t, k, v)
+                L.q.copy_(q)
+                L.candidates(t)                 # id lists built before the timed region
+                L.window_ids(t)
+                L.chunk_ids(t)
+            if t >= warm:
+                torch.cuda.synchronize()
+                a.record(s)
+            for L in layers:
+                L.step(t)
+            if t >= warm:
+                b.record(s)
+                times.append((a, b))
+        torch.cuda.synchronize()
+        ms = float(np.mean([a.elapsed_time(b) for a, b in times]))
+        kv = sum(layer_bytes(L) for L in layers)
+        dense_kv = w.n_chunks * w.nb_c * w.bs * w.D * 2 * 2 * w.B * w.H * w.layers
+        out[name] = {"layers": w.layers, "P": w.P, "policy": "merge_mean" if w.policy else "evict",
+                     "per_chunk_ms": round(ms, 4), "timed_steps": f"{warm}..{steps - 1}",
+                     "kv_bytes": kv, "dense_full_cache_kv_bytes_at_last_step": dense_kv,
+                     "kv_reduction": round(1 - kv / dense_kv, 4)}
+        del layers, pre
+        torch.cuda.empty_cache()
+    return out
+
+
 # ----------------------------------------------------------------- CPU oracle
 def cpu_oracle_sample(w, snap, n_heads=2, n_qblocks=None):
     """Time the oracle on a bounded sample: the full score/update/select on the
@@ -402,6 +554,12 @@ def main():
         line["e2e"] = {"value": round(world * flops / (e2e_ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
                        "ms_per_step": round(e2e_ms, 4), "h2d_bytes_per_step": h2d,
                        "d2h_bytes_per_step": d2h}
+    if world == 1 and not args.no_extras:
+        extras = {"dense_comparators_on_decode_inputs": bench_dense_comparators(torch, runner,
+                                                                                 runner.flush_buf)}
+        extras["train"] = bench_train(torch, runner.flush_buf)
+        extras["rollouts"] = bench_rollouts(torch)
+        line["extras"] = extras
     if rank == 0 and not args.no_cpu:
         fl, dt, desc = cpu_oracle_sample(w, runner.snap)
         line["cpu_baseline"] = {"value": round(fl / dt / 1e12, 6), "unit": "TFLOP/s",
