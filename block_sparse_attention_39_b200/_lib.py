@@ -22,6 +22,22 @@ class PbsaDims(ctypes.Structure):
 
 P = ctypes.POINTER(PbsaDims)
 
+# field order and types of pbsa_route_args (include/pbsa.h)
+ROUTE_FIELDS = [
+    ("q", c_void_p), ("Tq", c_int), ("kpool", c_void_p), ("vpool", c_void_p), ("NB", c_int),
+    ("blk_len", c_void_p), ("blk_pos", c_void_p), ("pool_ids", c_void_p), ("n_pool", c_int),
+    ("q_bar", c_void_p), ("k_bar", c_void_p), ("scores", c_void_p), ("mem_score", c_void_p),
+    ("P", c_int), ("n_sink", c_int), ("slot_src", c_void_p), ("slot_w", c_void_p),
+    ("cand_ids", c_void_p), ("cand_src", c_void_p), ("n_cand", c_int), ("policy", c_int),
+    ("win_ids", c_void_p), ("n_win", c_int), ("k", c_int), ("mem_ids", c_void_p),
+    ("n_mem", c_int), ("mask", c_int), ("q_pos0", c_int), ("idx", c_void_p), ("cnt", c_void_p),
+    ("Amax", c_int),
+]
+
+
+class PbsaRouteArgs(ctypes.Structure):
+    _fields_ = ROUTE_FIELDS
+
 # name -> (restype, argtypes); mirrors include/pbsa.h
 SIGNATURES = {
     "pbsa_score_blocks": (c_int, [P, c_void_p, c_int, c_void_p, c_int, c_void_p, c_void_p, c_int,
@@ -33,6 +49,8 @@ SIGNATURES = {
     "pbsa_select_local": (c_int, [P, c_void_p, c_int, c_int, c_void_p, c_int, c_int, c_void_p,
                                   c_int, c_int, c_void_p, c_int, c_int, c_void_p, c_int, c_void_p,
                                   c_void_p, c_int, c_int, c_int, c_void_p]),
+    "pbsa_route_workspace": (c_size_t, [P, c_int, c_int]),
+    "pbsa_route_step": (c_int, [P, ctypes.POINTER(PbsaRouteArgs), c_void_p, c_size_t, c_void_p]),
     "pbsa_attn_fwd": (c_int, [P, c_void_p, c_int, c_int, c_void_p, c_void_p, c_int, c_void_p,
                               c_void_p, c_void_p, c_void_p, c_int, c_int, c_void_p, c_void_p,
                               c_void_p]),

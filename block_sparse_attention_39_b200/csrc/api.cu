@@ -7,7 +7,10 @@
 #include <string>
 
 #include "common.cuh"
+#include "launch.h"
 #include "tmap.h"
+
+#include <cstdlib>
 
 namespace pbsa {
 
@@ -22,6 +25,27 @@ static int64_t g_wait_limit_ns = 2000000000LL;
 void set_error(const std::string& msg) { t_last_error = msg; }
 int debug_flags() { return g_debug_flags; }
 int64_t wait_limit_ns() { return g_wait_limit_ns; }
+
+bool pdl_enabled() {
+  static const bool on = [] {
+    const char* e = std::getenv("PBSA_PDL");
+    return !(e != nullptr && e[0] == '0');
+  }();
+  return on;
+}
+
+int sm_count() {
+  static int counts[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (counts[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1)
+      n = 148;
+    counts[dev] = n;
+  }
+  return counts[dev];
+}
 
 int* device_status_ptr() {
   static int* ptrs[64] = {nullptr};

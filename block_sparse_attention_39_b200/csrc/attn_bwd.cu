@@ -24,6 +24,7 @@
 #include <cuda_bf16.h>
 
 #include "common.cuh"
+#include "launch.h"
 #include "tc_sm100.cuh"
 #include "tmap.h"
 
@@ -59,6 +60,8 @@ struct BwdParams {
 // ------------------------------------------------------------------ prep
 template <int D>
 __global__ void __launch_bounds__(256) bwd_prep_kernel(BwdParams p) {
+  pdl_wait();
+  pdl_trigger();
   const int qi = blockIdx.x;
   const long bh = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -98,6 +101,8 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(BwdParams p) {
 // ------------------------------------------------------------------ reverse lists
 __global__ void __launch_bounds__(256) bwd_rev_kernel(BwdParams p) {
   __shared__ int part[256];
+  pdl_wait();
+  pdl_trigger();
   const long bh = blockIdx.x;
   const int t = threadIdx.x;
   const int per = (p.NB + 255) / 256;
@@ -176,6 +181,8 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                 const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                 BwdParams p) {
   using C = DkdvCfg<D>;
+  pdl_wait();
+  pdl_trigger();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -426,6 +433,8 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
               const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
               BwdParams p) {
   using C = DqCfg<D, NST>;
+  pdl_wait();
+  pdl_trigger();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -670,15 +679,16 @@ int launch_bwd(const pbsa_dims* d, BwdParams& p, const CUtensorMap& mq, const CU
   if (cudaMemsetAsync(static_cast<char*>(ws) + L.bitmap, 0, L.rev_off - L.bitmap, s) !=
       cudaSuccess)
     PBSA_CHECK_LAUNCH("attn_bwd: memset");
-  bwd_prep_kernel<D><<<dim3(p.nQB, BH), 256, 0, s>>>(p);
-  PBSA_CHECK_LAUNCH("bwd_prep_kernel");
-  bwd_rev_kernel<<<BH, 256, 0, s>>>(p);
-  PBSA_CHECK_LAUNCH("bwd_rev_kernel");
+  if (launch(bwd_prep_kernel<D>, dim3(p.nQB, BH), dim3(256), 0, s, p) != cudaSuccess)
+    PBSA_CHECK_LAUNCH("bwd_prep_kernel");
+  if (launch(bwd_rev_kernel, dim3(BH), dim3(256), 0, s, p) != cudaSuccess)
+    PBSA_CHECK_LAUNCH("bwd_rev_kernel");
   {
     auto kern = bwd_dkdv_kernel<D>;
     opt_in_smem<bwd_dkdv_kernel<D>>();
-    kern<<<static_cast<unsigned>(BH) * p.NB, 192, DkdvCfg<D>::SMEM, s>>>(mq, mdo, mk, mv, p);
-    PBSA_CHECK_LAUNCH("bwd_dkdv_kernel");
+    if (launch(kern, dim3(static_cast<unsigned>(BH) * p.NB), dim3(192), DkdvCfg<D>::SMEM, s, mq,
+               mdo, mk, mv, p) != cudaSuccess)
+      PBSA_CHECK_LAUNCH("bwd_dkdv_kernel");
   }
   {
     constexpr int NST = 2;
@@ -686,8 +696,9 @@ int launch_bwd(const pbsa_dims* d, BwdParams& p, const CUtensorMap& mq, const CU
     opt_in_smem<bwd_dq_kernel<D, NST>>();
     const size_t smem = DqCfg<D, NST>::smem_bytes(p.Amax);
     PBSA_CHECK_ARG(smem <= 227 * 1024, PBSA_ERR_SHAPE, "attn_bwd: Amax too large");
-    kern<<<static_cast<unsigned>(BH) * p.nQB, 192, smem, s>>>(mq, mdo, mk, mv, p);
-    PBSA_CHECK_LAUNCH("bwd_dq_kernel");
+    if (launch(kern, dim3(static_cast<unsigned>(BH) * p.nQB), dim3(192), smem, s, mq, mdo, mk, mv,
+               p) != cudaSuccess)
+      PBSA_CHECK_LAUNCH("bwd_dq_kernel");
   }
   return PBSA_OK;
 }

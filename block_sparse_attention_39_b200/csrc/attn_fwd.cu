@@ -31,6 +31,7 @@
 #include <cuda_bf16.h>
 
 #include "common.cuh"
+#include "launch.h"
 #include "tc_sm100.cuh"
 #include "tmap.h"
 
@@ -113,6 +114,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                 const __grid_constant__ CUtensorMap tmV, FwdParams p) {
   using C = FwdCfg<D, BS, NSK, NSV>;
+  pdl_wait();
+  pdl_trigger();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -512,8 +515,9 @@ int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& 
     if (dev >= 0 && dev < 64) opted[dev] = true;
   }
   const long tiles = static_cast<long>(prm.B) * prm.H * prm.nQB;
-  kern<<<static_cast<unsigned>(tiles), kFwdThreads, smem, s>>>(mq, mk, mv, prm);
-  PBSA_CHECK_LAUNCH("attn_fwd_kernel");
+  if (launch(kern, dim3(static_cast<unsigned>(tiles)), dim3(kFwdThreads), smem, s, mq, mk, mv,
+             prm) != cudaSuccess)
+    PBSA_CHECK_LAUNCH("attn_fwd_kernel");
   return PBSA_OK;
 }
 

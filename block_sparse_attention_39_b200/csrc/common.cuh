@@ -103,6 +103,17 @@ __device__ __forceinline__ void report_status(int* status, int code) {
   atomicCAS(status, 0, code);
 }
 
+// Programmatic dependent launch.  Every library kernel is launched with the
+// programmatic-serialisation attribute (see launch.h), so its CTAs may start
+// while the previous kernel on the stream is still running.  pdl_wait() blocks
+// until that kernel has completed and its memory is visible; every kernel calls
+// it before its first global-memory access.  pdl_trigger() lets the next
+// kernel's CTAs be scheduled once every CTA of this grid has started.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // Warp-wide bitonic sort of 32*KPL 64-bit keys, DESCENDING.  Element e of the
 // virtual array lives in lane (e / KPL), register (e % KPL).
 template <int KPL>

@@ -55,6 +55,9 @@ class PbsaLayer:
         self.max_cand = max(max_cand, 1)
         ws = K.update_memory_workspace(self.d, max(P, 1), self.max_cand)
         self.ws = torch.empty(ws, dtype=torch.uint8, device=dev)
+        # the fused routing call's workspace: barrier words (zero) + update plan
+        self.rws = torch.zeros(K.route_workspace(self.d, P, self.max_cand), dtype=torch.uint8,
+                               device=dev)
         self._ids = {}
         if self.tdtype != torch.bfloat16:
             # attention runs on bf16 copies of an fp32 cache (R17)
@@ -158,13 +161,35 @@ class PbsaLayer:
         cs = self.ids(key + ("src",), [g for c in chunks for g in w.chunk_global_ids(c)])
         return ci, cs
 
-    def step(self, t, stream=None):
-        """Score -> update -> select -> attend for chunk t (its Q already in self.q,
-        its K/V already in the pool)."""
-        self.score(t, stream=stream)
+    def route(self, t, stream=None):
+        """Score -> update -> select for chunk t in one call (pbsa_route_step)."""
+        w = self.w
+        pids = self.chunk_ids(t)
         ci, cs = self.candidates(t)
-        self.update(ci, cs, stream=stream)
-        self.select(t, stream=stream)
+        win = self.window_ids(t)
+        n_cand = ci.numel() if self.P else 0
+        K.route_step(self.d, self.rws, stream,
+                     q=self.q, Tq=w.chunk_tokens, kpool=self.kpool, vpool=self.vpool, NB=self.NB,
+                     blk_len=self.blk_len, blk_pos=self.blk_pos, pool_ids=pids,
+                     n_pool=pids.numel(), q_bar=self.q_bar, k_bar=self.k_bar, scores=self.scores,
+                     mem_score=self.mem, P=self.P, n_sink=w.n_sink,
+                     slot_src=self.slot_src if self.P else None,
+                     slot_w=self.slot_w if self.P else None,
+                     cand_ids=ci if n_cand else None, cand_src=cs if n_cand else None,
+                     n_cand=n_cand, policy=w.policy, win_ids=win, n_win=win.numel(), k=w.k,
+                     mem_ids=self.mem_ids, n_mem=self.P, mask=w.mask, q_pos0=t * w.chunk_tokens,
+                     idx=self.idx, cnt=self.cnt, Amax=self.Amax)
+
+    def step(self, t, stream=None, fused=True):
+        """Score -> update -> select -> attend for chunk t (its Q already in self.q,
+        its K/V already in the pool).  fused: the first three as one routing call."""
+        if fused:
+            self.route(t, stream=stream)
+        else:
+            self.score(t, stream=stream)
+            ci, cs = self.candidates(t)
+            self.update(ci, cs, stream=stream)
+            self.select(t, stream=stream)
         self.attend(t, stream=stream)
 
 

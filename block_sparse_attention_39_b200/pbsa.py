@@ -11,7 +11,7 @@ from typing import Optional
 
 import torch
 
-from ._lib import PbsaDims, lib
+from ._lib import ROUTE_FIELDS, PbsaDims, PbsaRouteArgs, lib
 
 BF16, FP32 = 0, 1
 EVICT, MERGE_MEAN = 0, 1
@@ -91,6 +91,31 @@ def select_local(d: PbsaDims, scores, nQB, NB, win_ids, n_win, k, mem_ids, n_mem
         ctypes.byref(d), _p(scores), nQB, NB, _p(win_ids), n_win, k, mp, n_mem, mem_ld,
         _p(blk_len), mask, q_pos0, _p(blk_pos), Tq, _p(idx), _p(cnt), Amax, qb_offset,
         nQB if nQB_total is None else nQB_total, _s(stream)))
+
+
+def route_workspace(d: PbsaDims, P: int, n_cand: int) -> int:
+    return int(lib().pbsa_route_workspace(ctypes.byref(d), P, n_cand))
+
+
+def route_step(d: PbsaDims, workspace, stream=None, **fields):
+    """pbsa_route_step: score -> update -> select in one call.  `fields` are the
+    members of pbsa_route_args (tensors for pointers, ints otherwise); members
+    not given are NULL / 0.  The first 256 bytes of `workspace` must be zero
+    before the first call (torch.zeros does it)."""
+    args = PbsaRouteArgs()
+    names = {n for n, _ in ROUTE_FIELDS}
+    for name, val in fields.items():
+        if name not in names:
+            raise TypeError(f"pbsa_route_args has no member {name!r}")
+        if isinstance(val, torch.Tensor):
+            setattr(args, name, _p(val))
+        elif val is None:
+            setattr(args, name, None)
+        else:
+            setattr(args, name, int(val))
+    _check("pbsa_route_step", lib().pbsa_route_step(
+        ctypes.byref(d), ctypes.byref(args), _p(workspace),
+        workspace.numel() * workspace.element_size(), _s(stream)))
 
 
 def attn_fwd(d: PbsaDims, q, Tq, q_pos0, kpool, vpool, NB, blk_len, blk_pos, idx, cnt, Amax, mask,

@@ -175,6 +175,75 @@ int pbsa_select_local(const pbsa_dims* dims, const float* scores, int nQB, int N
                       int qb_offset, int nQB_total, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * a1..a5 in one launch: score -> update memory -> select for one query chunk.
+ * Passages: those of pbsa_score_blocks, pbsa_update_memory and
+ * pbsa_select_local above; this call has no separate counterpart on the pages.
+ * It is the routing half of a decode step as the pages order it.
+ *
+ * Results are exactly those of the three calls made in order on the same
+ * stream:
+ *   pbsa_score_blocks(dims, q, Tq, kpool, NB, blk_len, pool_ids, n_pool,
+ *                     q_bar, k_bar, scores, mem_score)
+ *   pbsa_update_memory(dims, kpool, vpool, NB, blk_len, blk_pos, k_bar, P,
+ *                      n_sink, slot_src, slot_w, cand_ids, cand_src, n_cand,
+ *                      mem_score, policy, ...)   -- skipped if P == 0 or n_cand == 0
+ *   pbsa_select_local(dims, scores, nQB, NB, win_ids, n_win, k, mem_ids, n_mem,
+ *                     0, blk_len, mask, q_pos0, blk_pos, Tq, idx, cnt, Amax,
+ *                     0, nQB)
+ * with the same argument rules and limits.  The work runs as one cooperative
+ * kernel (phases separated by grid barriers) when the shape has an
+ * instantiation (n_win <= 256 and n_mem + min(k, n_win) <= 128) and a
+ * co-resident grid; otherwise the call makes the three per-call launches
+ * itself.
+ *
+ * workspace: device, 256-byte aligned, at least pbsa_route_workspace() bytes.
+ * Its first 256 bytes hold the grid barrier's counters: zero them once before
+ * the first call (e.g. cudaMemset); every call leaves them zero again.  The
+ * rest is the update's workspace.  Calls that share a workspace must not run
+ * concurrently.
+ * ------------------------------------------------------------------------- */
+typedef struct {
+  /* a1 + a2 */
+  const void* q;
+  int Tq;
+  void* kpool;
+  void* vpool;
+  int NB;
+  int32_t* blk_len;
+  int32_t* blk_pos;
+  const int32_t* pool_ids;
+  int n_pool;
+  float* q_bar;
+  float* k_bar;
+  float* scores;
+  float* mem_score;
+  /* a3 */
+  int P;
+  int n_sink;
+  int32_t* slot_src;
+  float* slot_w;
+  const int32_t* cand_ids;
+  const int32_t* cand_src;
+  int n_cand;
+  int policy; /* pbsa_policy */
+  /* a4 + a5 */
+  const int32_t* win_ids;
+  int n_win;
+  int k;
+  const int32_t* mem_ids;
+  int n_mem;
+  int mask; /* pbsa_mask */
+  int q_pos0;
+  int32_t* idx;
+  int32_t* cnt;
+  int Amax;
+} pbsa_route_args;
+
+size_t pbsa_route_workspace(const pbsa_dims* dims, int P, int n_cand);
+int pbsa_route_step(const pbsa_dims* dims, const pbsa_route_args* args, void* workspace,
+                    size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
  * a6: hybrid block-sparse attention, forward.
  * Passage: gist.science/es section 2 PBSA item "Atención Híbrida" (dense over
  * the persistent memory plus sparse over the local window, one kernel) and

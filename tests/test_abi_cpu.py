@@ -105,3 +105,42 @@ def test_select_limits():
     # window too long for one warp
     assert lib.pbsa_select_local(ctypes.byref(d), fake, 1, 600, fake, 600, 16, NULL, 0, 0, fake, 0,
                                  0, NULL, 100, fake, fake, 64, 0, 1, NULL) == -2
+
+
+def test_route_args_layout_matches_the_header(tmp_path):
+    # the ctypes mirror of pbsa_route_args must have the C layout: compile a
+    # probe against the header with the host compiler and compare offsets
+    fields = [n for n, _ in _lib.ROUTE_FIELDS]
+    src = tmp_path / "layout.c"
+    src.write_text('#include <stdio.h>\n#include <stddef.h>\n#include "pbsa.h"\nint main(void){\n'
+                   + "".join(f'  printf("%zu\\n", offsetof(pbsa_route_args, {n}));\n' for n in fields)
+                   + '  printf("%zu\\n", sizeof(pbsa_route_args));\n  return 0;\n}\n')
+    exe = tmp_path / "layout"
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no host C compiler")
+    subprocess.run([cc, "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)], check=True)
+    got = [int(x) for x in subprocess.run([str(exe)], check=True, capture_output=True,
+                                          text=True).stdout.split()]
+    want = [getattr(_lib.PbsaRouteArgs, n).offset for n in fields] + [ctypes.sizeof(_lib.PbsaRouteArgs)]
+    assert got == want
+
+
+def test_route_rejects_bad_arguments_without_launch():
+    lib = _lib.lib()
+    d = _d()
+    assert lib.pbsa_route_step(ctypes.byref(d), None, None, 0, None) == -1
+    a = _lib.PbsaRouteArgs(Tq=128, NB=8, n_pool=0, P=0, n_cand=0)
+    # no workspace
+    assert lib.pbsa_route_step(ctypes.byref(d), ctypes.byref(a), None, 0, None) == -7
+    # workspace too small: the barrier words alone need 256 bytes
+    assert lib.pbsa_route_step(ctypes.byref(d), ctypes.byref(a), ctypes.c_void_p(4096), 128,
+                               None) == -7
+    a.Tq = 0
+    assert lib.pbsa_route_step(ctypes.byref(d), ctypes.byref(a), ctypes.c_void_p(4096), 4096,
+                               None) == -2
+    assert lib.pbsa_route_workspace(ctypes.byref(d), 0, 0) == 256
+    assert (lib.pbsa_route_workspace(ctypes.byref(d), 24, 111)
+            == 256 + lib.pbsa_update_memory_workspace(ctypes.byref(d), 24, 111))
