@@ -101,11 +101,14 @@ __global__ void __launch_bounds__(kRouteThreads, 2) route_kernel(RouteParams r) 
                       static_cast<const T*>(r.vpool), static_cast<T*>(const_cast<void*>(r.stash)));
       grid_sync(r, target += G);
     }
+    int* s_mref = reinterpret_cast<int*>(smem + 8 * D * sizeof(float));
+    int* s_mlen = s_mref + kMaxItems;
+    float* s_mw = reinterpret_cast<float*>(s_mlen + kMaxItems);
     for (int it = cta; it < n_slot_items; it += G)
       apply_item<T, D>(r.upd, it % r.P, it / r.P, static_cast<T*>(r.kpool),
                        static_cast<T*>(r.vpool), static_cast<const T*>(r.stash), r.blk_len,
                        r.blk_pos, r.k_bar, r.slot_src, r.slot_w,
-                       reinterpret_cast<float(*)[D]>(smem));
+                       reinterpret_cast<float(*)[D]>(smem), s_mref, s_mlen, s_mw);
     grid_sync(r, target += G);
   }
 
@@ -137,9 +140,9 @@ size_t route_smem(const RouteParams& r) {
   m = std::max(m, score_smem_bytes<D>(r.nQB));
   if (r.do_update) {
     size_t plan = (sizeof(PlanSmem) + 15) / 16 * 16;
-    if (r.upd.policy == PBSA_MERGE_MEAN) plan += static_cast<size_t>(r.P) * D * sizeof(float);
+    if (r.upd.policy == PBSA_MERGE_MEAN) plan += merge_key_smem(r.P, D);
     m = std::max(m, plan);
-    m = std::max(m, static_cast<size_t>(8) * D * sizeof(float));
+    m = std::max(m, static_cast<size_t>(8) * D * sizeof(float) + 3 * kMaxItems * sizeof(int));
   }
   return m;
 }

@@ -37,10 +37,12 @@ update_apply_kernel(UpdArgs a, T* __restrict__ kpool, T* __restrict__ vpool,
                     int32_t* __restrict__ blk_pos, float* __restrict__ k_bar,
                     int32_t* __restrict__ slot_src, float* __restrict__ slot_w) {
   __shared__ float red[8][D];
+  __shared__ int s_mref[kMaxItems], s_mlen[kMaxItems];
+  __shared__ float s_mw[kMaxItems];
   pdl_wait();
   pdl_trigger();
   apply_item<T, D>(a, static_cast<int>(blockIdx.x), blockIdx.y, kpool, vpool, stash, blk_len,
-                   blk_pos, k_bar, slot_src, slot_w, red);
+                   blk_pos, k_bar, slot_src, slot_w, red, s_mref, s_mlen, s_mw);
 }
 
 template <typename T, int D>
@@ -107,15 +109,14 @@ extern "C" int pbsa_update_memory(const pbsa_dims* d, void* kpool, void* vpool, 
   a.slot_w = slot_w; a.cand_ids = cand_ids; a.cand_src = cand_src; a.mem = mem_score;
   a.ws = workspace; a.status = status;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const size_t plan_smem =
-      policy == PBSA_MERGE_MEAN ? static_cast<size_t>(P) * d->D * sizeof(float) : 0;
+  const size_t plan_smem = policy == PBSA_MERGE_MEAN ? merge_key_smem(P, d->D) : 0;
   {
     static bool attr_set[64] = {false};
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev >= 0 && dev < 64 && !attr_set[dev]) {
       cudaFuncSetAttribute(update_plan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           256 * 128 * 4);
+                           static_cast<int>(merge_key_smem(256, 128)));
       attr_set[dev] = true;
     }
   }

@@ -110,6 +110,12 @@ __device__ __forceinline__ int block_excl_scan256(int v, int* tot, int* total) {
 }
 
 // --------------------------------------------------------------------- plan
+// Dynamic shared memory of plan_head under the merge policy: the kept slots'
+// pooled keys (padded rows) and one loser key per warp.
+__host__ __device__ inline size_t merge_key_smem(int P, int D) {
+  return (static_cast<size_t>(P) * (D / 4 + 1) + 8 * static_cast<size_t>(D / 4)) * 16;
+}
+
 // Shared memory of plan_head (one (b,h) at a time, 256 threads).
 struct PlanSmem {
   uint64_t skey[kMaxItems];
@@ -232,21 +238,41 @@ __device__ inline void plan_head(const UpdArgs& a, long bh, PlanSmem& sm, float*
     if (f) free_pos[at] = t;
   }
   __syncthreads();
-  // newly kept blocks take free slots in ascending global-id order
-  if (t < NI && it_rank[t] >= 0 && it_rank[t] < n_keep && it_old[t] < 0) {
-    int r = 0;
-    for (int u = 0; u < NI; ++u)
-      if (it_rank[u] >= 0 && it_rank[u] < n_keep && it_old[u] < 0 && it_src[u] < it_src[t]) ++r;
-    it_slot[t] = free_pos[r];
-    holder[free_pos[r]] = t;
+  // newly kept blocks take free slots in ascending global-id order.  When the
+  // candidates' global ids ascend with their list position (the usual case:
+  // a chunk's blocks in order), that order is the item order and a prefix
+  // count gives each block its free slot; otherwise every block counts the
+  // kept new blocks with smaller ids.
+  {
+    const bool is_new_kept = t < NI && it_rank[t] >= 0 && it_rank[t] < n_keep && it_old[t] < 0;
+    const bool ascending =
+        __syncthreads_and(!(t > n_dyn && t < NI && it_src[t - 1] >= it_src[t])) != 0;
+    if (ascending) {
+      const int r = block_excl_scan256(is_new_kept ? 1 : 0, s_tot, nullptr);
+      if (is_new_kept) {
+        it_slot[t] = free_pos[r];
+        holder[free_pos[r]] = t;
+      }
+    } else if (is_new_kept) {
+      int r = 0;
+      for (int u = 0; u < NI; ++u)
+        if (it_rank[u] >= 0 && it_rank[u] < n_keep && it_old[u] < 0 && it_src[u] < it_src[t]) ++r;
+      it_slot[t] = free_pos[r];
+      holder[free_pos[r]] = t;
+    }
   }
   __syncthreads();
 
-  // ---- merge targets: most similar kept slot by pooled-key dot product.
-  // The kept blocks' pooled keys are staged in shared memory first.
+  // ---- merge targets: most similar kept slot by pooled-key dot product
+  // (ties -> lowest slot).  The kept blocks' pooled keys are staged in shared
+  // memory with a padded row stride; each warp takes one loser at a time, its
+  // lanes take one slot each (a full dot product over D, in dimension order),
+  // and a warp argmax picks the target.
   if (a.policy == PBSA_MERGE_MEAN && n_keep > 0) {
     const int D4 = a.D / 4;
-    float4* sk4 = reinterpret_cast<float4*>(sk);
+    const int ST4 = D4 + 1;                          // padded row stride (float4)
+    float4* sk4 = reinterpret_cast<float4*>(sk);     // [P][ST4]
+    float4* kw = sk4 + P * ST4 + warp * D4;          // this warp's loser key
     const float4* kb4 = reinterpret_cast<const float4*>(a.k_bar);
     for (int e0 = 0; e0 < P * D4; e0 += 256 * 4) {
       float4 v[4];
@@ -260,43 +286,67 @@ __device__ inline void plan_head(const UpdArgs& a, long bh, PlanSmem& sm, float*
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
         const int e = e0 + q * 256 + t;
-        if (e < P * D4) sk4[e] = v[q];
+        if (e < P * D4) sk4[(e / D4) * ST4 + e % D4] = v[q];
       }
     }
     __syncthreads();
     for (int u = warp; u < NI; u += 8) {
       if (!(it_rank[u] >= n_keep)) continue;          // losers only (warp-uniform)
-      const float* kj = a.k_bar + (bh * a.NB + it_phys[u]) * static_cast<long>(a.D);
-      float kjr[4];
-#pragma unroll
-      for (int q = 0; q < 4; ++q) kjr[q] = lane + 32 * q < a.D ? kj[lane + 32 * q] : 0.f;
+      if (lane < D4) kw[lane] = kb4[(bh * a.NB + it_phys[u]) * D4 + lane];
+      __syncwarp();
       float best = -INFINITY;
       int best_s = -1;
-      for (int s = n_sink; s < P; ++s) {
-        const int c = holder[s];
-        if (c < 0) continue;
-        const float* kc = sk + s * a.D;
-        float part = 0.f;
+      for (int s0 = n_sink; s0 < P; s0 += 32) {
+        const int s = s0 + lane;
+        const bool valid = s < P && holder[s] >= 0;
+        float dot = 0.f;
+        if (s < P) {
+          const float4* kc = sk4 + s * ST4;
+          for (int d4 = 0; d4 < D4; ++d4) {
+            const float4 x = kw[d4], y = kc[d4];
+            dot = fmaf(x.x, y.x, dot);
+            dot = fmaf(x.y, y.y, dot);
+            dot = fmaf(x.z, y.z, dot);
+            dot = fmaf(x.w, y.w, dot);
+          }
+        }
+        float v = valid ? dot : -INFINITY;
+        int si = valid ? s : 0x7fffffff;
 #pragma unroll
-        for (int q = 0; q < 4; ++q)
-          if (lane + 32 * q < a.D) part = fmaf(kjr[q], kc[lane + 32 * q], part);
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
-        if (part > best || best_s < 0) { best = part; best_s = s; }
+        for (int off = 16; off > 0; off >>= 1) {
+          const float ov = __shfl_xor_sync(0xffffffffu, v, off);
+          const int os = __shfl_xor_sync(0xffffffffu, si, off);
+          if (ov > v || (ov == v && os < si)) {
+            v = ov;
+            si = os;
+          }
+        }
+        if (si != 0x7fffffff && (v > best || best_s < 0)) {
+          best = v;
+          best_s = si;
+        }
       }
       if (lane == 0) it_target[u] = best_s;
+      __syncwarp();
     }
   }
   // merge lists grouped by target slot, each in ranking order (deterministic
-  // summation order): a counting sort over the losers
-  if (t < P) tcount[t] = 0;
+  // summation order): the losers are listed by rank, then one warp per target
+  // slot counts (and later places) its losers with ballots
+  const bool merging = a.policy == PBSA_MERGE_MEAN && n_keep > 0;
+  const int n_lose = n_valid - n_keep;
+  int* rank_item = free_pos;                 // free_pos is no longer needed
+  if (merging && t < NI && it_rank[t] >= n_keep) rank_item[it_rank[t] - n_keep] = t;
   __syncthreads();
-  int my_pos = 0;
-  const int my_target = (t < NI) ? it_target[t] : -1;
-  if (my_target >= 0) {
-    atomicAdd(&tcount[my_target], 1);
-    for (int u = 0; u < NI; ++u)
-      if (it_target[u] == my_target && it_rank[u] < it_rank[t]) ++my_pos;
+  for (int s = warp; s < P; s += 8) {
+    int n = 0;
+    if (merging) {
+      for (int c0 = 0; c0 < n_lose; c0 += 32) {
+        const int u = c0 + lane < n_lose ? rank_item[c0 + lane] : -1;
+        n += __popc(__ballot_sync(0xffffffffu, u >= 0 && it_target[u] == s));
+      }
+    }
+    if (lane == 0) tcount[s] = n;
   }
   __syncthreads();
 
@@ -337,13 +387,24 @@ __device__ inline void plan_head(const UpdArgs& a, long bh, PlanSmem& sm, float*
   if (t < NI && it_target[t] >= 0 && it_old[t] >= 0 && s_op[it_old[t]] == OP_WRITE)
     pv.stash[it_old[t]] = 1;
   __syncthreads();
-  if (my_target >= 0) {
-    const int slot = s_moff[my_target] + my_pos;
-    const int old = it_old[t];
-    const bool from_stash = old >= 0 && s_op[old] == OP_WRITE;
-    pv.mref[slot] = from_stash ? -(1 + old) : it_phys[t];
-    pv.mlen[slot] = it_len[t];
-    pv.mw[slot] = it_w[t];
+  if (merging) {
+    for (int s = warp; s < P; s += 8) {
+      int base = s_moff[s];
+      for (int c0 = 0; c0 < n_lose; c0 += 32) {
+        const int u = c0 + lane < n_lose ? rank_item[c0 + lane] : -1;
+        const bool hit = u >= 0 && it_target[u] == s;
+        const unsigned m = __ballot_sync(0xffffffffu, hit);
+        if (hit) {
+          const int slot = base + __popc(m & ((1u << lane) - 1u));
+          const int old = it_old[u];
+          const bool from_stash = old >= 0 && s_op[old] == OP_WRITE;
+          pv.mref[slot] = from_stash ? -(1 + old) : it_phys[u];
+          pv.mlen[slot] = it_len[u];
+          pv.mw[slot] = it_w[u];
+        }
+        base += __popc(m);
+      }
+    }
   }
 }
 
@@ -385,6 +446,13 @@ struct Elem<__nv_bfloat16> {
     x[0] = bf16_lo(u.x); x[1] = bf16_hi(u.x); x[2] = bf16_lo(u.y); x[3] = bf16_hi(u.y);
     x[4] = bf16_lo(u.z); x[5] = bf16_hi(u.z); x[6] = bf16_lo(u.w); x[7] = bf16_hi(u.w);
   }
+  __device__ static uint4 raw(const __nv_bfloat16* p) { return *reinterpret_cast<const uint4*>(p); }
+  __device__ static void fma_raw(float w, uint4 u, float (&acc)[8]) {
+    acc[0] = fmaf(w, bf16_lo(u.x), acc[0]); acc[1] = fmaf(w, bf16_hi(u.x), acc[1]);
+    acc[2] = fmaf(w, bf16_lo(u.y), acc[2]); acc[3] = fmaf(w, bf16_hi(u.y), acc[3]);
+    acc[4] = fmaf(w, bf16_lo(u.z), acc[4]); acc[5] = fmaf(w, bf16_hi(u.z), acc[5]);
+    acc[6] = fmaf(w, bf16_lo(u.w), acc[6]); acc[7] = fmaf(w, bf16_hi(u.w), acc[7]);
+  }
   // rounds to storage, stores, and returns the stored values in x
   __device__ static void store(__nv_bfloat16* p, float (&x)[8]) {
     uint4 u;
@@ -402,19 +470,26 @@ struct Elem<float> {
     float4 u = *reinterpret_cast<const float4*>(p);
     x[0] = u.x; x[1] = u.y; x[2] = u.z; x[3] = u.w;
   }
+  __device__ static uint4 raw(const float* p) { return *reinterpret_cast<const uint4*>(p); }
+  __device__ static void fma_raw(float w, uint4 u, float (&acc)[4]) {
+    acc[0] = fmaf(w, __uint_as_float(u.x), acc[0]); acc[1] = fmaf(w, __uint_as_float(u.y), acc[1]);
+    acc[2] = fmaf(w, __uint_as_float(u.z), acc[2]); acc[3] = fmaf(w, __uint_as_float(u.w), acc[3]);
+  }
   __device__ static void store(float* p, float (&x)[4]) {
     *reinterpret_cast<float4*>(p) = make_float4(x[0], x[1], x[2], x[3]);
   }
 };
 
 // Write slot s of head bh as planned (copy, weighted mean or clear) and update
-// its pooled key and metadata.  `red` holds 8*D floats.
+// its pooled key and metadata.  `red` holds 8*D floats; s_mref, s_mlen and
+// s_mw are shared arrays of kMaxItems entries for the slot's merge list.
 template <typename T, int D>
 __device__ void apply_item(const UpdArgs& a, int s, long bh, T* __restrict__ kpool,
                            T* __restrict__ vpool, const T* __restrict__ stash,
                            int32_t* __restrict__ blk_len, int32_t* __restrict__ blk_pos,
                            float* __restrict__ k_bar, int32_t* __restrict__ slot_src,
-                           float* __restrict__ slot_w, float (*red)[D]) {
+                           float* __restrict__ slot_w, float (*red)[D], int* s_mref,
+                           int* s_mlen, float* s_mw) {
   constexpr int EPC = Elem<T>::EPC;
   constexpr int CPR = D / EPC;
   constexpr int RPP = 256 / CPR;
@@ -478,35 +553,51 @@ __device__ void apply_item(const UpdArgs& a, int s, long bh, T* __restrict__ kpo
     }
     return;
   }
-  // weighted row-wise mean of the base and its merged losers
+  // weighted row-wise mean of the base and its merged losers.  The merge list
+  // is read into shared memory once; rows are processed RG row passes at a
+  // time so that all loads of one merge source are in flight together.
+  const int nm = m1 - m0;
+  for (int m = t; m < nm; m += 256) {
+    s_mref[m] = pv.mref[m0 + m];
+    s_mlen[m] = pv.mlen[m0 + m];
+    s_mw[m] = pv.mw[m0 + m];
+  }
+  __syncthreads();
   float wsum = bw;
   int nlen = blen;
-  for (int m = m0; m < m1; ++m) {
-    wsum += pv.mw[m];
-    nlen = max(nlen, pv.mlen[m]);
+  for (int m = 0; m < nm; ++m) {
+    wsum += s_mw[m];
+    nlen = max(nlen, s_mlen[m]);
   }
   const float inv = 1.f / wsum;
   const int c = t % CPR, rg = t / CPR;
+  constexpr int RG = 2;
   float colsum[EPC];
 #pragma unroll
   for (int e = 0; e < EPC; ++e) colsum[e] = 0.f;
-  for (int r = rg; r < a.bs; r += RPP) {
-    const long off = static_cast<long>(r) * D + c * EPC;
-    float ak[EPC], av[EPC], x[EPC];
+  for (int r0 = rg; r0 < a.bs; r0 += RG * RPP) {
+    float ak[RG][EPC], av[RG][EPC];
 #pragma unroll
-    for (int e = 0; e < EPC; ++e) { ak[e] = 0.f; av[e] = 0.f; }
-    if (r < blen) {
-      Elem<T>::load(kb + off, x);
+    for (int i = 0; i < RG; ++i) {
+      const int r = r0 + i * RPP;
+      const long off = static_cast<long>(r) * D + c * EPC;
+      float xk[EPC], xv[EPC];
 #pragma unroll
-      for (int e = 0; e < EPC; ++e) ak[e] = bw * x[e];
-      Elem<T>::load(vb + off, x);
+      for (int e = 0; e < EPC; ++e) { xk[e] = 0.f; xv[e] = 0.f; }
+      if (r < a.bs && r < blen) {
+        Elem<T>::load(kb + off, xk);
+        Elem<T>::load(vb + off, xv);
+      }
 #pragma unroll
-      for (int e = 0; e < EPC; ++e) av[e] = bw * x[e];
+      for (int e = 0; e < EPC; ++e) {
+        ak[i][e] = r < blen ? bw * xk[e] : 0.f;
+        av[i][e] = r < blen ? bw * xv[e] : 0.f;
+      }
     }
-    for (int m = m0; m < m1; ++m) {
-      if (r >= pv.mlen[m]) continue;
-      const int ref = pv.mref[m];
-      const float w = pv.mw[m];
+    for (int m = 0; m < nm; ++m) {
+      const int ref = s_mref[m];
+      const int ml = s_mlen[m];
+      const float w = s_mw[m];
       const T* ks;
       const T* vs;
       if (ref >= 0) {
@@ -517,21 +608,39 @@ __device__ void apply_item(const UpdArgs& a, int s, long bh, T* __restrict__ kpo
         ks = stash + ((bh * a.P + so) * 2 + 0) * blk_elems;
         vs = stash + ((bh * a.P + so) * 2 + 1) * blk_elems;
       }
-      Elem<T>::load(ks + off, x);
+      uint4 xk[RG], xv[RG];
 #pragma unroll
-      for (int e = 0; e < EPC; ++e) ak[e] = fmaf(w, x[e], ak[e]);
-      Elem<T>::load(vs + off, x);
+      for (int i = 0; i < RG; ++i) {
+        const int r = r0 + i * RPP;
+        if (r < a.bs && r < ml) {
+          const long off = static_cast<long>(r) * D + c * EPC;
+          xk[i] = Elem<T>::raw(ks + off);
+          xv[i] = Elem<T>::raw(vs + off);
+        }
+      }
 #pragma unroll
-      for (int e = 0; e < EPC; ++e) av[e] = fmaf(w, x[e], av[e]);
+      for (int i = 0; i < RG; ++i) {
+        const int r = r0 + i * RPP;
+        if (r < a.bs && r < ml) {
+          Elem<T>::fma_raw(w, xk[i], ak[i]);
+          Elem<T>::fma_raw(w, xv[i], av[i]);
+        }
+      }
     }
 #pragma unroll
-    for (int e = 0; e < EPC; ++e) { ak[e] *= inv; av[e] *= inv; }
-    // every thread reads its own elements above before writing them here
-    Elem<T>::store(kd + off, ak);
-    Elem<T>::store(vd + off, av);
-    if (r < nlen) {
+    for (int i = 0; i < RG; ++i) {
+      const int r = r0 + i * RPP;
+      if (r >= a.bs) continue;
+      const long off = static_cast<long>(r) * D + c * EPC;
 #pragma unroll
-      for (int e = 0; e < EPC; ++e) colsum[e] += ak[e];
+      for (int e = 0; e < EPC; ++e) { ak[i][e] *= inv; av[i][e] *= inv; }
+      // every thread reads its own elements above before writing them here
+      Elem<T>::store(kd + off, ak[i]);
+      Elem<T>::store(vd + off, av[i]);
+      if (r < nlen) {
+#pragma unroll
+        for (int e = 0; e < EPC; ++e) colsum[e] += ak[i][e];
+      }
     }
   }
 #pragma unroll
