@@ -136,21 +136,22 @@ __global__ void __launch_bounds__(256) bwd_rev_kernel(BwdParams p) {
   if (t == 255) roff[p.NB] = part[255];
 }
 
-// ------------------------------------------------------------------ shared
-// Write 8 consecutive bf16 (columns 8q..8q+7 of row `row`) of a 128-row,
-// K-major, 128-byte-swizzled operand tile made of 64-column atoms.
-__device__ __forceinline__ void st_sw128_chunk(uint8_t* tile, int row, int col8, uint4 v) {
-  const int atom = col8 >> 3;          // 8 chunks of 8 columns per atom
-  const int q = col8 & 7;
-  uint8_t* dst = tile + atom * (128 * 128) + row * 128 + ((q ^ (row & 7)) << 4);
-  *reinterpret_cast<uint4*>(dst) = v;
-}
-
-__device__ __forceinline__ void fence_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
 // ------------------------------------------------------------------ dK / dV
+// One CTA per key block j (the 128-row tiles K_j and V_j stay in shared
+// memory), iterating over the query blocks i that attend it, in ascending
+// order.  Q_i, dO_i and the rows' LSE and Delta stream through two stages.
+// Tensor memory:
+//   TM_ST   S^T = K_j Q_i^T (fp32).  The softmax warps overwrite its first 64
+//           columns with P^T (bf16 pairs): the A operand of dV += P^T dO_i.
+//   TM_DPT  dP^T = V_j dO_i^T.  Overwritten by dS^T = P^T (dP^T - Delta) (bf16
+//           pairs): the A operand of dK += dS^T Q_i.
+//   TM_DV, TM_DK  the accumulators.
+// The MMA warp issues dV_i, S^T_{i+1}, dK_i, dP^T_{i+1} in that order: the
+// tensor cores compute the next query block's S^T while the softmax warps
+// form dS^T_i, and every reuse of a TMEM region is safe because tcgen05 MMAs
+// issued by one thread run in order.  Thread c of the four softmax warps owns
+// key row c (TMEM lane c) and keeps its 128 probabilities in registers between
+// the P^T and dS^T passes.
 template <int D>
 struct DkdvCfg {
   static constexpr int KB = D / 64;
@@ -158,17 +159,14 @@ struct DkdvCfg {
   static constexpr int TILE = KB * BOX;            // one 128-row operand tile
   static constexpr int OFF_K = 0;
   static constexpr int OFF_V = OFF_K + TILE;
-  static constexpr int OFF_Q = OFF_V + TILE;
-  static constexpr int OFF_DO = OFF_Q + TILE;
-  static constexpr int OFF_PT = OFF_DO + TILE;     // P^T, 128 x 128 bf16
-  static constexpr int OFF_DST = OFF_PT + 2 * BOX; // dS^T
-  static constexpr int OFF_LSE = OFF_DST + 2 * BOX;  // [2][128] floats
+  static constexpr int OFF_Q = OFF_V + TILE;       // 2 stages
+  static constexpr int OFF_DO = OFF_Q + 2 * TILE;  // 2 stages
+  static constexpr int OFF_LSE = OFF_DO + 2 * TILE;  // [2][128] floats (log2 units)
   static constexpr int OFF_DL = OFF_LSE + 2 * 128 * 4;
   static constexpr int OFF_BAR = OFF_DL + 2 * 128 * 4;
-  // barriers
-  static constexpr int B_KV = 0, B_QF = 1, B_QE = 2, B_SF = 3, B_PF = 4, B_DSF = 5, B_MMA = 6;
-  static constexpr int B_ST = 7;   // + parity (2): LSE/Delta staged by all 128 row threads
-  static constexpr int NBAR = 9;
+  static constexpr int B_KV = 0, B_QF = 1, B_QE = 3, B_SF = 5, B_DPF = 6, B_PF = 7, B_DSF = 8,
+                       B_MMA = 9;
+  static constexpr int NBAR = 10;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int SMEM = 1024 + OFF_MISC + 16;
   static constexpr int TM_ST = 0, TM_DPT = 128, TM_DV = 256, TM_DK = 256 + D;
@@ -197,7 +195,6 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
 
   const uint32_t sK = smem_u32(smem + C::OFF_K), sV = smem_u32(smem + C::OFF_V);
   const uint32_t sQ = smem_u32(smem + C::OFF_Q), sDO = smem_u32(smem + C::OFF_DO);
-  const uint32_t sPT = smem_u32(smem + C::OFF_PT), sDST = smem_u32(smem + C::OFF_DST);
   float* s_lse = reinterpret_cast<float*>(smem + C::OFF_LSE);
   float* s_dl = reinterpret_cast<float*>(smem + C::OFF_DL);
   const uint32_t bar0 = smem_u32(smem + C::OFF_BAR);
@@ -207,14 +204,15 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
 
   if (tid == 0) {
     mbar_init(BAR(C::B_KV), 1);
-    mbar_init(BAR(C::B_QF), 1);
-    mbar_init(BAR(C::B_QE), 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(BAR(C::B_QF + s), 1);
+      mbar_init(BAR(C::B_QE + s), 1);
+    }
     mbar_init(BAR(C::B_SF), 1);
-    mbar_init(BAR(C::B_PF), 128);
-    mbar_init(BAR(C::B_DSF), 128);
+    mbar_init(BAR(C::B_DPF), 1);
+    mbar_init(BAR(C::B_PF), 4);    // one arrival per softmax warp
+    mbar_init(BAR(C::B_DSF), 4);
     mbar_init(BAR(C::B_MMA), 1);
-    mbar_init(BAR(C::B_ST), 128);
-    mbar_init(BAR(C::B_ST + 1), 128);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -228,140 +226,182 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   const uint32_t tmem = *tmem_holder;
 
   if (warp == 4) {
-    if (lane == 0 && n > 0) {
-      const int kv_row = (bh * p.NB + j) * p.bs;
-      mbar_expect_tx(BAR(C::B_KV), 2 * C::TILE);
-#pragma unroll
-      for (int kb = 0; kb < C::KB; ++kb) {
-        tma_load_2d(sK + kb * C::BOX, &tmK, BAR(C::B_KV), kb * 64, kv_row);
-        tma_load_2d(sV + kb * C::BOX, &tmV, BAR(C::B_KV), kb * 64, kv_row);
-      }
+    // ---------------------------------------------------------- producer
+    // K_j, V_j once; per query block: its LSE and Delta staged by the 32
+    // lanes, then Q_i and dO_i by TMA into stage i & 1.
+    if (n > 0) {
       int issued = 0;
-      for (int it = 0; it < n; ++it) {
-        if (it > 0 && !mbar_wait(BAR(C::B_QE), (it - 1) & 1, abort_flag, p.status, p.limit_ns))
-          break;
-        int qrow0, qlen;
-        qb_rows(rq[it], p.Tq, p.q_chunk, p.bs, qrow0, qlen);
-        const int q_row = bh * p.Tq + qrow0;
-        mbar_expect_tx(BAR(C::B_QF), 2 * C::TILE);
+      if (lane == 0) {
+        const int kv_row = (bh * p.NB + j) * p.bs;
+        mbar_expect_tx(BAR(C::B_KV), 2 * C::TILE);
 #pragma unroll
         for (int kb = 0; kb < C::KB; ++kb) {
-          tma_load_2d(sQ + kb * C::BOX, &tmQ, BAR(C::B_QF), kb * 64, q_row);
-          tma_load_2d(sDO + kb * C::BOX, &tmDO, BAR(C::B_QF), kb * 64, q_row);
+          tma_load_2d(sK + kb * C::BOX, &tmK, BAR(C::B_KV), kb * 64, kv_row);
+          tma_load_2d(sV + kb * C::BOX, &tmV, BAR(C::B_KV), kb * 64, kv_row);
+        }
+      }
+      for (int it = 0; it < n; ++it) {
+        const int s = it & 1;
+        bool ok = true;
+        if (it >= 2)
+          ok = mbar_wait(BAR(C::B_QE + s), ((it >> 1) & 1) ^ 1, abort_flag, p.status, p.limit_ns);
+        if (!__all_sync(0xffffffffu, ok)) break;
+        int qrow0, qlen;
+        qb_rows(rq[it], p.Tq, p.q_chunk, p.bs, qrow0, qlen);
+        const long row_base = static_cast<long>(bh) * p.Tq + qrow0;
+        for (int r = lane; r < 128; r += 32) {
+          float l2 = INFINITY, dl = 0.f;
+          if (r < qlen) {
+            const float lse = p.lse[row_base + r];
+            l2 = lse == -INFINITY ? INFINITY : lse * 1.4426950408889634f;
+            dl = p.delta[row_base + r];
+          }
+          s_lse[s * 128 + r] = l2;
+          s_dl[s * 128 + r] = dl;
+        }
+        __syncwarp();
+        if (lane == 0) {
+          mbar_expect_tx(BAR(C::B_QF + s), 2 * C::TILE);   // release: LSE/Delta staged
+#pragma unroll
+          for (int kb = 0; kb < C::KB; ++kb) {
+            tma_load_2d(sQ + s * C::TILE + kb * C::BOX, &tmQ, BAR(C::B_QF + s), kb * 64,
+                        static_cast<int>(row_base));
+            tma_load_2d(sDO + s * C::TILE + kb * C::BOX, &tmDO, BAR(C::B_QF + s), kb * 64,
+                        static_cast<int>(row_base));
+          }
         }
         issued = it + 1;
       }
-      mbar_drain(BAR(C::B_KV), 0, p.status, p.limit_ns);
-      if (issued > 0) mbar_drain(BAR(C::B_QF), (issued - 1) & 1, p.status, p.limit_ns);
+      if (lane == 0) {
+        mbar_drain(BAR(C::B_KV), 0, p.status, p.limit_ns);
+        for (int it = max(0, issued - 2); it < issued; ++it)
+          mbar_drain(BAR(C::B_QF + (it & 1)), (it >> 1) & 1, p.status, p.limit_ns);
+      }
     }
     __syncwarp();
   } else if (warp == 5) {
+    // ---------------------------------------------------------- MMA issuer
     if (lane == 0 && n > 0) {
       constexpr uint32_t id_kk = idesc_bf16_f32(128, 128, false, false);  // K-major x K-major
       constexpr uint32_t id_kmn = idesc_bf16_f32(128, D, false, true);    // B MN-major
-      if (mbar_wait(BAR(C::B_KV), 0, abort_flag, p.status, p.limit_ns)) {
-        for (int it = 0; it < n; ++it) {
-          if (!mbar_wait(BAR(C::B_QF), it & 1, abort_flag, p.status, p.limit_ns)) break;
-          tc_fence_after();
+      auto issue_st = [&](int it) -> bool {   // S^T_it = K Q_it^T
+        const int s = it & 1;
+        if (!mbar_wait(BAR(C::B_QF + s), (it >> 1) & 1, abort_flag, p.status, p.limit_ns))
+          return false;
+        tc_fence_after();
 #pragma unroll
-          for (int k = 0; k < D / 16; ++k) {
-            const uint32_t off = (k >> 2) * C::BOX + (k & 3) * 32;
-            mma_ss(tmem + C::TM_ST, smem_desc_sw128(sK + off, 16, 1024),
-                   smem_desc_sw128(sQ + off, 16, 1024), id_kk, k > 0);
-            mma_ss(tmem + C::TM_DPT, smem_desc_sw128(sV + off, 16, 1024),
-                   smem_desc_sw128(sDO + off, 16, 1024), id_kk, k > 0);
-          }
-          mma_commit(BAR(C::B_SF));
-          if (!mbar_wait(BAR(C::B_PF), it & 1, abort_flag, p.status, p.limit_ns)) break;
-          tc_fence_after();
-#pragma unroll
-          for (int k = 0; k < 128 / 16; ++k) {
-            const uint32_t aoff = (k >> 2) * C::BOX + (k & 3) * 32;
-            mma_ss(tmem + C::TM_DV, smem_desc_sw128(sPT + aoff, 16, 1024),
-                   smem_desc_sw128(sDO + k * 2048, C::BOX, 1024), id_kmn, (it > 0 || k > 0));
-          }
-          if (!mbar_wait(BAR(C::B_DSF), it & 1, abort_flag, p.status, p.limit_ns)) break;
-          tc_fence_after();
-#pragma unroll
-          for (int k = 0; k < 128 / 16; ++k) {
-            const uint32_t aoff = (k >> 2) * C::BOX + (k & 3) * 32;
-            mma_ss(tmem + C::TM_DK, smem_desc_sw128(sDST + aoff, 16, 1024),
-                   smem_desc_sw128(sQ + k * 2048, C::BOX, 1024), id_kmn, (it > 0 || k > 0));
-          }
-          mma_commit(BAR(C::B_QE));
+        for (int k = 0; k < D / 16; ++k) {
+          const uint32_t off = (k >> 2) * C::BOX + (k & 3) * 32;
+          mma_ss(tmem + C::TM_ST, smem_desc_sw128(sK + off, 16, 1024),
+                 smem_desc_sw128(sQ + s * C::TILE + off, 16, 1024), id_kk, k > 0);
         }
+        mma_commit(BAR(C::B_SF));
+        return true;
+      };
+      auto issue_dpt = [&](int it) {          // dP^T_it = V dO_it^T (Q/dO stage already full)
+        const int s = it & 1;
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k) {
+          const uint32_t off = (k >> 2) * C::BOX + (k & 3) * 32;
+          mma_ss(tmem + C::TM_DPT, smem_desc_sw128(sV + off, 16, 1024),
+                 smem_desc_sw128(sDO + s * C::TILE + off, 16, 1024), id_kk, k > 0);
+        }
+        mma_commit(BAR(C::B_DPF));
+      };
+      bool ok = mbar_wait(BAR(C::B_KV), 0, abort_flag, p.status, p.limit_ns) && issue_st(0);
+      if (ok) issue_dpt(0);
+      for (int it = 0; ok && it < n; ++it) {
+        const int s = it & 1;
+        if (!mbar_wait(BAR(C::B_PF), it & 1, abort_flag, p.status, p.limit_ns)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int k = 0; k < 128 / 16; ++k)        // dV += P^T dO_it
+          mma_ts(tmem + C::TM_DV, tmem + C::TM_ST + k * 8,
+                 smem_desc_sw128(sDO + s * C::TILE + k * 2048, C::BOX, 1024), id_kmn,
+                 (it > 0 || k > 0) ? 1u : 0u);
+        if (it + 1 < n && !issue_st(it + 1)) break;
+        if (!mbar_wait(BAR(C::B_DSF), it & 1, abort_flag, p.status, p.limit_ns)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int k = 0; k < 128 / 16; ++k)        // dK += dS^T Q_it
+          mma_ts(tmem + C::TM_DK, tmem + C::TM_DPT + k * 8,
+                 smem_desc_sw128(sQ + s * C::TILE + k * 2048, C::BOX, 1024), id_kmn,
+                 (it > 0 || k > 0) ? 1u : 0u);
+        mma_commit(BAR(C::B_QE + s));
+        if (it + 1 < n) issue_dpt(it + 1);
       }
       mma_commit(BAR(C::B_MMA));
       mbar_drain(BAR(C::B_MMA), 0, p.status, p.limit_ns);
     }
     __syncwarp();
   } else {
-    // ---------------------------------------------------------- row warps
+    // ---------------------------------------------------------- softmax rows
     const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
-    const int c = tid;                      // key row in the tile
+    const int c = tid;                      // key row of the tile
+    const bool row_ok = c < klen;
     bool ok = true;
     for (int it = 0; it < n; ++it) {
-      const int qi = rq[it];
+      const int s = it & 1;
       int qrow0, qlen;
-      qb_rows(qi, p.Tq, p.q_chunk, p.bs, qrow0, qlen);
-      float* lse_b = s_lse + (it & 1) * 128;
-      float* dl_b = s_dl + (it & 1) * 128;
-      {
-        const int r = tid;
-        float l2 = INFINITY, dl = 0.f;
-        if (r < qlen) {
-          const float lse = p.lse[static_cast<long>(bh) * p.Tq + qrow0 + r];
-          l2 = lse == -INFINITY ? INFINITY : lse * 1.4426950408889634f;
-          dl = p.delta[static_cast<long>(bh) * p.Tq + qrow0 + r];
-        }
-        lse_b[r] = l2;
-        dl_b[r] = dl;
-      }
-      // every row thread needs all 128 staged values: bounded handshake
-      mbar_arrive(BAR(C::B_ST + (it & 1)));
-      ok = mbar_wait(BAR(C::B_ST + (it & 1)), (it >> 1) & 1, abort_flag, p.status, p.limit_ns);
-      ok = __all_sync(0xffffffffu, ok);
-      if (!ok) break;
-      ok = mbar_wait(BAR(C::B_SF), it & 1, abort_flag, p.status, p.limit_ns);
+      qb_rows(rq[it], p.Tq, p.q_chunk, p.bs, qrow0, qlen);
+      // stage s is full (LSE/Delta visible), then S^T_it is in TMEM
+      ok = mbar_wait(BAR(C::B_QF + s), (it >> 1) & 1, abort_flag, p.status, p.limit_ns) &&
+           mbar_wait(BAR(C::B_SF), it & 1, abort_flag, p.status, p.limit_ns);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
+      const float* lse_b = s_lse + s * 128;
+      const float* dl_b = s_dl + s * 128;
       const int qpos0 = p.q_pos0 + qrow0;
-      const bool row_ok = c < klen;
-#pragma unroll 1
+      // first visible query column of this key row (rows past qlen have LSE = +inf)
+      const int r_min = !row_ok ? 1 << 20
+                                : (p.mask == PBSA_MASK_TOKEN ? max(0, kpos0 + c - qpos0) : 0);
+      float P[128];
+#pragma unroll
       for (int cc = 0; cc < 4; ++cc) {
-        uint32_t sv[32], dv[32];
+        uint32_t sv[32];
         tmem_ld32(tmem + lane_base + C::TM_ST + cc * 32, sv);
+        tmem_wait_ld();
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          // visible columns are r >= r_min; the exponent always runs (ex2(-inf) = 0)
+          const int r = cc * 32 + e;
+          const float x = __uint_as_float(sv[e]) * p.scale_log2 - lse_b[r];
+          P[r] = ex2(r >= r_min ? x : -INFINITY);
+        }
+#pragma unroll
+        for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(P[cc * 32 + 2 * e], P[cc * 32 + 2 * e + 1]);
+        // columns [16cc, 16cc + 16) of S^T were read by this chunk or the one before
+        tmem_st16(tmem + lane_base + C::TM_ST + cc * 16, pk);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(BAR(C::B_PF));
+      ok = mbar_wait(BAR(C::B_DPF), it & 1, abort_flag, p.status, p.limit_ns);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after();
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) {
+        uint32_t dv[32];
         tmem_ld32(tmem + lane_base + C::TM_DPT + cc * 32, dv);
         tmem_wait_ld();
-        uint32_t pk[16], dk[16];
+        uint32_t dk[16];
 #pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          float pv[2], ds[2];
-#pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            const int r = cc * 32 + e + u;
-            bool vis = row_ok && r < p.bs;
-            if (p.mask == PBSA_MASK_TOKEN) vis = vis && (kpos0 + c <= qpos0 + r);
-            const float x = __uint_as_float(sv[e + u]) * p.scale_log2 - lse_b[r];
-            pv[u] = vis ? ex2(x) : 0.f;
-            ds[u] = pv[u] * (__uint_as_float(dv[e + u]) - dl_b[r]);
-          }
-          pk[e >> 1] = pack_bf16x2(pv[0], pv[1]);
-          dk[e >> 1] = pack_bf16x2(ds[0], ds[1]);
+        for (int e = 0; e < 16; ++e) {
+          const int r = cc * 32 + 2 * e;
+          const float d0 = P[r] * (__uint_as_float(dv[2 * e]) - dl_b[r]);
+          const float d1 = P[r + 1] * (__uint_as_float(dv[2 * e + 1]) - dl_b[r + 1]);
+          dk[e] = pack_bf16x2(d0, d1);
         }
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          st_sw128_chunk(smem + C::OFF_PT, c, cc * 4 + q,
-                         make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]));
-          st_sw128_chunk(smem + C::OFF_DST, c, cc * 4 + q,
-                         make_uint4(dk[4 * q], dk[4 * q + 1], dk[4 * q + 2], dk[4 * q + 3]));
-        }
+        tmem_st16(tmem + lane_base + C::TM_DPT + cc * 16, dk);
       }
-      fence_async_smem();
+      tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(BAR(C::B_PF));
-      mbar_arrive(BAR(C::B_DSF));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(BAR(C::B_DSF));
     }
     // ---------------------------------------------------------- epilogue
     if (ok && n > 0) {
@@ -407,7 +447,18 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
 }
 
 // ------------------------------------------------------------------ dQ
-template <int D, int NST>
+// One CTA per query block (Q and dO stay in shared memory), iterating over its
+// attended key blocks; K_j streams through NK stages and V_j through NV
+// stages (K is needed until dQ_j, V only until dP_j).  Tensor memory:
+//   TM_S0, TM_S1  S_j = Q K_j^T for alternate j; the softmax warps read S_j,
+//                 keep P_j in registers and later overwrite S_j's first 64
+//                 columns with dS_j = P_j (dP_j - Delta) (bf16 pairs): the A
+//                 operand of dQ += dS_j K_j;
+//   TM_DP         dP_j = dO V_j^T;
+//   TM_DQ         the accumulator.
+// The MMA warp issues dQ_j, dP_{j+1}, S_{j+2}: S_{j+1} is already computed
+// when the softmax warps finish block j.
+template <int D, int NK, int NV>
 struct DqCfg {
   static constexpr int KB = D / 64;
   static constexpr int BOX = 128 * 128;
@@ -415,24 +466,24 @@ struct DqCfg {
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_DO = OFF_Q + TILE;
   static constexpr int OFF_K = OFF_DO + TILE;
-  static constexpr int OFF_V = OFF_K + NST * TILE;
-  static constexpr int OFF_BAR = OFF_V + NST * TILE;
-  static constexpr int B_Q = 0, B_KF = 1, B_VF = 1 + NST, B_KVE = 1 + 2 * NST;
-  static constexpr int B_SF = 1 + 3 * NST, B_DSF = 2 + 3 * NST, B_MMA = 3 + 3 * NST;
-  static constexpr int NBAR = 4 + 3 * NST;
+  static constexpr int OFF_V = OFF_K + NK * TILE;
+  static constexpr int OFF_BAR = OFF_V + NV * TILE;
+  static constexpr int B_Q = 0, B_KF = 1, B_KE = 1 + NK, B_VF = 1 + 2 * NK, B_VE = 1 + 2 * NK + NV,
+                       B_SF = 1 + 2 * NK + 2 * NV, B_DPF = B_SF + 2, B_DSF = B_DPF + 1,
+                       B_MMA = B_DSF + 1;
+  static constexpr int NBAR = B_MMA + 1;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
-  static constexpr int OFF_IDS = OFF_MISC + 16;
-  static constexpr int TM_S = 0, TM_DP = 128, TM_DQ = 256, TM_DS = 256 + D;
+  static constexpr int SMEM = 1024 + OFF_MISC + 16;
+  static constexpr int TM_S0 = 0, TM_DP = 128, TM_DQ = 256, TM_S1 = 256 + D;
   static constexpr int TM_COLS = 512;
-  static size_t smem_bytes(int Amax) { return 1024 + OFF_IDS + 3 * 4 * static_cast<size_t>(Amax); }
 };
 
-template <int D, int NST>
+template <int D, int NK, int NV>
 __global__ void __launch_bounds__(192, 1)
 bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmDO,
               const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
               BwdParams p) {
-  using C = DqCfg<D, NST>;
+  using C = DqCfg<D, NK, NV>;
   pdl_wait();
   pdl_trigger();
   extern __shared__ uint8_t smem_raw[];
@@ -445,6 +496,7 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
   n = max(0, min(n, p.Amax));
   int qrow0, qlen;
   qb_rows(qi, p.Tq, p.q_chunk, p.bs, qrow0, qlen);
+  const int32_t* row_ids = p.idx + (static_cast<long>(bh) * p.nQB + qi) * p.Amax;
 
   const uint32_t sQ = smem_u32(smem + C::OFF_Q), sDO = smem_u32(smem + C::OFF_DO);
   const uint32_t sK = smem_u32(smem + C::OFF_K), sV = smem_u32(smem + C::OFF_V);
@@ -452,37 +504,24 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
   auto BAR = [&](int k) { return bar0 + 8u * static_cast<uint32_t>(k); };
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
-  int* s_ids = reinterpret_cast<int*>(smem + C::OFF_IDS);
-  int* s_len = s_ids + p.Amax;
-  int* s_pos = s_len + p.Amax;
 
   if (tid == 0) {
     mbar_init(BAR(C::B_Q), 1);
-    for (int s = 0; s < NST; ++s) {
+    for (int s = 0; s < NK; ++s) {
       mbar_init(BAR(C::B_KF + s), 1);
+      mbar_init(BAR(C::B_KE + s), 1);
+    }
+    for (int s = 0; s < NV; ++s) {
       mbar_init(BAR(C::B_VF + s), 1);
-      mbar_init(BAR(C::B_KVE + s), 1);
+      mbar_init(BAR(C::B_VE + s), 1);
     }
     mbar_init(BAR(C::B_SF), 1);
-    mbar_init(BAR(C::B_DSF), 128);
+    mbar_init(BAR(C::B_SF + 1), 1);
+    mbar_init(BAR(C::B_DPF), 1);
+    mbar_init(BAR(C::B_DSF), 4);    // one arrival per softmax warp
     mbar_init(BAR(C::B_MMA), 1);
     *abort_flag = 0;
     fence_mbar_init();
-  }
-  const int32_t* row_ids = p.idx + (static_cast<long>(bh) * p.nQB + qi) * p.Amax;
-  for (int e = tid; e < n; e += blockDim.x) {
-    int id = row_ids[e];
-    int len = 0, pos = 0;
-    if (id < 0 || id >= p.NB) {
-      report_status(p.status, PBSA_ERR_ARG);
-      id = 0;
-    } else {
-      len = min(max(p.blk_len[static_cast<long>(bh) * p.NB + id], 0), p.bs);
-      pos = p.blk_pos ? p.blk_pos[static_cast<long>(bh) * p.NB + id] : 0;
-    }
-    s_ids[e] = id;
-    s_len[e] = len;
-    s_pos[e] = pos;
   }
   if (warp == 4) {
     tmem_alloc(smem_u32(tmem_holder), C::TM_COLS);
@@ -493,7 +532,19 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
 
+  // physical id of attended block jj (an invalid id is reported and read as
+  // block 0, fully masked)
+  auto block_id = [&](int jj) -> int {
+    const int id = row_ids[jj];
+    if (id < 0 || id >= p.NB) {
+      report_status(p.status, PBSA_ERR_ARG);
+      return -1;
+    }
+    return id;
+  };
+
   if (warp == 4) {
+    // ---------------------------------------------------------- producer
     if (lane == 0 && n > 0) {
       const int q_row = bh * p.Tq + qrow0;
       mbar_expect_tx(BAR(C::B_Q), 2 * C::TILE);
@@ -502,65 +553,94 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         tma_load_2d(sQ + kb * C::BOX, &tmQ, BAR(C::B_Q), kb * 64, q_row);
         tma_load_2d(sDO + kb * C::BOX, &tmDO, BAR(C::B_Q), kb * 64, q_row);
       }
-      int issued = 0;
+      int k_issued = 0, v_issued = 0;
       for (int jj = 0; jj < n; ++jj) {
-        const int s = jj % NST;
-        if (jj >= NST &&
-            !mbar_wait(BAR(C::B_KVE + s), ((jj / NST) & 1) ^ 1, abort_flag, p.status, p.limit_ns))
+        const int id = max(block_id(jj), 0);
+        const int kv_row = (bh * p.NB + id) * p.bs;
+        const int ks = jj % NK, vs = jj % NV;
+        if (jj >= NK &&
+            !mbar_wait(BAR(C::B_KE + ks), ((jj / NK) & 1) ^ 1, abort_flag, p.status, p.limit_ns))
           break;
-        const int kv_row = (bh * p.NB + s_ids[jj]) * p.bs;
-        mbar_expect_tx(BAR(C::B_KF + s), C::TILE);
+        mbar_expect_tx(BAR(C::B_KF + ks), C::TILE);
 #pragma unroll
         for (int kb = 0; kb < C::KB; ++kb)
-          tma_load_2d(sK + s * C::TILE + kb * C::BOX, &tmK, BAR(C::B_KF + s), kb * 64, kv_row);
-        mbar_expect_tx(BAR(C::B_VF + s), C::TILE);
+          tma_load_2d(sK + ks * C::TILE + kb * C::BOX, &tmK, BAR(C::B_KF + ks), kb * 64, kv_row);
+        k_issued = jj + 1;
+        if (jj >= NV &&
+            !mbar_wait(BAR(C::B_VE + vs), ((jj / NV) & 1) ^ 1, abort_flag, p.status, p.limit_ns))
+          break;
+        mbar_expect_tx(BAR(C::B_VF + vs), C::TILE);
 #pragma unroll
         for (int kb = 0; kb < C::KB; ++kb)
-          tma_load_2d(sV + s * C::TILE + kb * C::BOX, &tmV, BAR(C::B_VF + s), kb * 64, kv_row);
-        issued = jj + 1;
+          tma_load_2d(sV + vs * C::TILE + kb * C::BOX, &tmV, BAR(C::B_VF + vs), kb * 64, kv_row);
+        v_issued = jj + 1;
       }
       mbar_drain(BAR(C::B_Q), 0, p.status, p.limit_ns);
-      for (int s = 0; s < NST && s < issued; ++s) {
-        const int jl = s + ((issued - 1 - s) / NST) * NST;
-        mbar_drain(BAR(C::B_KF + s), (jl / NST) & 1, p.status, p.limit_ns);
-        mbar_drain(BAR(C::B_VF + s), (jl / NST) & 1, p.status, p.limit_ns);
-      }
+      for (int jj = max(0, k_issued - NK); jj < k_issued; ++jj)
+        mbar_drain(BAR(C::B_KF + jj % NK), (jj / NK) & 1, p.status, p.limit_ns);
+      for (int jj = max(0, v_issued - NV); jj < v_issued; ++jj)
+        mbar_drain(BAR(C::B_VF + jj % NV), (jj / NV) & 1, p.status, p.limit_ns);
     }
     __syncwarp();
   } else if (warp == 5) {
+    // ---------------------------------------------------------- MMA issuer
     if (lane == 0 && n > 0) {
       constexpr uint32_t id_kk = idesc_bf16_f32(128, 128, false, false);
       constexpr uint32_t id_kmn = idesc_bf16_f32(128, D, false, true);
-      if (mbar_wait(BAR(C::B_Q), 0, abort_flag, p.status, p.limit_ns)) {
-        for (int jj = 0; jj < n; ++jj) {
-          const int s = jj % NST;
-          if (!mbar_wait(BAR(C::B_KF + s), (jj / NST) & 1, abort_flag, p.status, p.limit_ns)) break;
-          if (!mbar_wait(BAR(C::B_VF + s), (jj / NST) & 1, abort_flag, p.status, p.limit_ns)) break;
-          tc_fence_after();
+      auto issue_s = [&](int jj) -> bool {    // S_jj = Q K_jj^T
+        const int ks = jj % NK;
+        if (!mbar_wait(BAR(C::B_KF + ks), (jj / NK) & 1, abort_flag, p.status, p.limit_ns))
+          return false;
+        tc_fence_after();
+        const uint32_t d_tm = tmem + ((jj & 1) ? C::TM_S1 : C::TM_S0);
 #pragma unroll
-          for (int k = 0; k < D / 16; ++k) {
-            const uint32_t off = (k >> 2) * C::BOX + (k & 3) * 32;
-            mma_ss(tmem + C::TM_S, smem_desc_sw128(sQ + off, 16, 1024),
-                   smem_desc_sw128(sK + s * C::TILE + off, 16, 1024), id_kk, k > 0);
-            mma_ss(tmem + C::TM_DP, smem_desc_sw128(sDO + off, 16, 1024),
-                   smem_desc_sw128(sV + s * C::TILE + off, 16, 1024), id_kk, k > 0);
-          }
-          mma_commit(BAR(C::B_SF));
-          if (!mbar_wait(BAR(C::B_DSF), jj & 1, abort_flag, p.status, p.limit_ns)) break;
-          tc_fence_after();
-#pragma unroll
-          for (int k = 0; k < 128 / 16; ++k)
-            mma_ts(tmem + C::TM_DQ, tmem + C::TM_DS + k * 8,
-                   smem_desc_sw128(sK + s * C::TILE + k * 2048, C::BOX, 1024), id_kmn,
-                   (jj > 0 || k > 0));
-          mma_commit(BAR(C::B_KVE + s));
+        for (int k = 0; k < D / 16; ++k) {
+          const uint32_t off = (k >> 2) * C::BOX + (k & 3) * 32;
+          mma_ss(d_tm, smem_desc_sw128(sQ + off, 16, 1024),
+                 smem_desc_sw128(sK + ks * C::TILE + off, 16, 1024), id_kk, k > 0);
         }
+        mma_commit(BAR(C::B_SF + (jj & 1)));
+        return true;
+      };
+      auto issue_dp = [&](int jj) -> bool {   // dP_jj = dO V_jj^T; frees V stage
+        const int vs = jj % NV;
+        if (!mbar_wait(BAR(C::B_VF + vs), (jj / NV) & 1, abort_flag, p.status, p.limit_ns))
+          return false;
+        tc_fence_after();
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k) {
+          const uint32_t off = (k >> 2) * C::BOX + (k & 3) * 32;
+          mma_ss(tmem + C::TM_DP, smem_desc_sw128(sDO + off, 16, 1024),
+                 smem_desc_sw128(sV + vs * C::TILE + off, 16, 1024), id_kk, k > 0);
+        }
+        mma_commit(BAR(C::B_DPF));
+        mma_commit(BAR(C::B_VE + vs));
+        return true;
+      };
+      bool ok = mbar_wait(BAR(C::B_Q), 0, abort_flag, p.status, p.limit_ns) && issue_s(0) &&
+                issue_dp(0) && (n < 2 || issue_s(1));
+      for (int jj = 0; ok && jj < n; ++jj) {
+        if (!mbar_wait(BAR(C::B_DSF), jj & 1, abort_flag, p.status, p.limit_ns)) break;
+        tc_fence_after();
+        const int ks = jj % NK;
+        const uint32_t ds_tm = tmem + ((jj & 1) ? C::TM_S1 : C::TM_S0);
+#pragma unroll
+        for (int k = 0; k < 128 / 16; ++k)        // dQ += dS_jj K_jj
+          mma_ts(tmem + C::TM_DQ, ds_tm + k * 8,
+                 smem_desc_sw128(sK + ks * C::TILE + k * 2048, C::BOX, 1024), id_kmn,
+                 (jj > 0 || k > 0) ? 1u : 0u);
+        mma_commit(BAR(C::B_KE + ks));
+        // dP_{jj+1} overwrites dP_jj (read by the softmax before DSF_jj);
+        // S_{jj+2} overwrites dS_jj (read by the dQ MMA just issued)
+        if (jj + 1 < n && !issue_dp(jj + 1)) break;
+        if (jj + 2 < n && !issue_s(jj + 2)) break;
       }
       mma_commit(BAR(C::B_MMA));
       mbar_drain(BAR(C::B_MMA), 0, p.status, p.limit_ns);
     }
     __syncwarp();
   } else {
+    // ---------------------------------------------------------- softmax rows
     const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
     const int r = tid;
     const bool row_ok = r < qlen;
@@ -571,39 +651,68 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       dl = p.delta[static_cast<long>(bh) * p.Tq + qrow0 + r];
     }
     const int qpos = p.q_pos0 + qrow0 + r;
+    // length and position of block jj, fetched one block ahead
+    auto meta = [&](int jj, int& len, int& pos) {
+      len = 0;
+      pos = 0;
+      if (jj < n) {
+        const int id = block_id(jj);
+        if (id >= 0) {
+          len = min(max(p.blk_len[static_cast<long>(bh) * p.NB + id], 0), p.bs);
+          pos = p.blk_pos ? p.blk_pos[static_cast<long>(bh) * p.NB + id] : 0;
+        }
+      }
+    };
+    int len_n, pos_n;
+    meta(0, len_n, pos_n);
     bool ok = true;
     for (int jj = 0; jj < n; ++jj) {
-      ok = mbar_wait(BAR(C::B_SF), jj & 1, abort_flag, p.status, p.limit_ns);
+      const int len = len_n, kpos0 = pos_n;
+      meta(jj + 1, len_n, pos_n);
+      ok = mbar_wait(BAR(C::B_SF + (jj & 1)), (jj >> 1) & 1, abort_flag, p.status, p.limit_ns);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
-      const int len = s_len[jj];
-      const int kpos0 = s_pos[jj];
-#pragma unroll 1
+      const uint32_t s_tm = tmem + lane_base + ((jj & 1) ? C::TM_S1 : C::TM_S0);
+      int c_lim = row_ok ? len : 0;
+      if (p.mask == PBSA_MASK_TOKEN) c_lim = min(c_lim, max(0, qpos - kpos0 + 1));
+      float P[128];
+#pragma unroll
       for (int cc = 0; cc < 4; ++cc) {
-        uint32_t sv[32], dv[32];
-        tmem_ld32(tmem + lane_base + C::TM_S + cc * 32, sv);
+        uint32_t sv[32];
+        tmem_ld32(s_tm + cc * 32, sv);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          // visible columns are col < c_lim; the exponent always runs (ex2(-inf) = 0)
+          const int col = cc * 32 + e;
+          const float x = __uint_as_float(sv[e]) * p.scale_log2 - l2;
+          P[col] = ex2(col < c_lim ? x : -INFINITY);
+        }
+      }
+      ok = mbar_wait(BAR(C::B_DPF), jj & 1, abort_flag, p.status, p.limit_ns);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after();
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) {
+        uint32_t dv[32];
         tmem_ld32(tmem + lane_base + C::TM_DP + cc * 32, dv);
         tmem_wait_ld();
         uint32_t pk[16];
 #pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          float ds[2];
-#pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            const int col = cc * 32 + e + u;
-            bool vis = row_ok && col < len;
-            if (p.mask == PBSA_MASK_TOKEN) vis = vis && (kpos0 + col <= qpos);
-            const float pv = vis ? ex2(__uint_as_float(sv[e + u]) * p.scale_log2 - l2) : 0.f;
-            ds[u] = pv * (__uint_as_float(dv[e + u]) - dl);
-          }
-          pk[e >> 1] = pack_bf16x2(ds[0], ds[1]);
+        for (int e = 0; e < 16; ++e) {
+          const int col = cc * 32 + 2 * e;
+          pk[e] = pack_bf16x2(P[col] * (__uint_as_float(dv[2 * e]) - dl),
+                              P[col + 1] * (__uint_as_float(dv[2 * e + 1]) - dl));
         }
-        tmem_st16(tmem + lane_base + C::TM_DS + cc * 16, pk);
+        // every column of S_jj was read above
+        tmem_st16(s_tm + cc * 16, pk);
       }
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(BAR(C::B_DSF));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(BAR(C::B_DSF));
     }
     if (ok && n > 0) {
       ok = mbar_wait(BAR(C::B_MMA), 0, abort_flag, p.status, p.limit_ns);
@@ -639,6 +748,7 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     tmem_dealloc(tmem, C::TM_COLS);
   }
 }
+
 
 struct BwdLayout {
   size_t delta, bitmap, rev_off, rev_q, total;
@@ -691,11 +801,11 @@ int launch_bwd(const pbsa_dims* d, BwdParams& p, const CUtensorMap& mq, const CU
       PBSA_CHECK_LAUNCH("bwd_dkdv_kernel");
   }
   {
-    constexpr int NST = 2;
-    auto kern = bwd_dq_kernel<D, NST>;
-    opt_in_smem<bwd_dq_kernel<D, NST>>();
-    const size_t smem = DqCfg<D, NST>::smem_bytes(p.Amax);
-    PBSA_CHECK_ARG(smem <= 227 * 1024, PBSA_ERR_SHAPE, "attn_bwd: Amax too large");
+    constexpr int NK = 3, NV = 2;
+    auto kern = bwd_dq_kernel<D, NK, NV>;
+    opt_in_smem<bwd_dq_kernel<D, NK, NV>>();
+    const size_t smem = DqCfg<D, NK, NV>::SMEM;
+    static_assert(DqCfg<128, 3, 2>::SMEM <= 227 * 1024, "dQ tiles exceed shared memory");
     if (launch(kern, dim3(static_cast<unsigned>(BH) * p.nQB), dim3(192), smem, s, mq, mdo, mk, mv,
                p) != cudaSuccess)
       PBSA_CHECK_LAUNCH("bwd_dq_kernel");
