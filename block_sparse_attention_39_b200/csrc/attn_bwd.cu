@@ -340,10 +340,16 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     const int c = tid;                      // key row of the tile
     const bool row_ok = c < klen;
     bool ok = true;
+    const bool tok = p.mask == PBSA_MASK_TOKEN;
+    int q_next = (tok && n > 0) ? rq[0] : 0;     // query block of the next step (token mask only)
     for (int it = 0; it < n; ++it) {
       const int s = it & 1;
-      int qrow0, qlen;
-      qb_rows(rq[it], p.Tq, p.q_chunk, p.bs, qrow0, qlen);
+      int qrow0 = 0;
+      if (tok) {
+        int qlen_unused;
+        qb_rows(q_next, p.Tq, p.q_chunk, p.bs, qrow0, qlen_unused);
+        if (it + 1 < n) q_next = rq[it + 1];
+      }
       // stage s is full (LSE/Delta visible), then S^T_it is in TMEM
       ok = mbar_wait(BAR(C::B_QF + s), (it >> 1) & 1, abort_flag, p.status, p.limit_ns) &&
            mbar_wait(BAR(C::B_SF), it & 1, abort_flag, p.status, p.limit_ns);
@@ -354,20 +360,26 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       const float* dl_b = s_dl + s * 128;
       const int qpos0 = p.q_pos0 + qrow0;
       // first visible query column of this key row (rows past qlen have LSE = +inf)
-      const int r_min = !row_ok ? 1 << 20
-                                : (p.mask == PBSA_MASK_TOKEN ? max(0, kpos0 + c - qpos0) : 0);
+      const int r_min = !row_ok ? 1 << 20 : (tok ? max(0, kpos0 + c - qpos0) : 0);
       float P[128];
 #pragma unroll
       for (int cc = 0; cc < 4; ++cc) {
         uint32_t sv[32];
         tmem_ld32(tmem + lane_base + C::TM_ST + cc * 32, sv);
+        // the 32 LSE values of this chunk: eight 128-bit broadcast reads
+        float lv[32];
+#pragma unroll
+        for (int v = 0; v < 8; ++v) {
+          const float4 t4 = reinterpret_cast<const float4*>(lse_b + cc * 32)[v];
+          lv[4 * v] = t4.x; lv[4 * v + 1] = t4.y; lv[4 * v + 2] = t4.z; lv[4 * v + 3] = t4.w;
+        }
         tmem_wait_ld();
         uint32_t pk[16];
 #pragma unroll
         for (int e = 0; e < 32; ++e) {
           // visible columns are r >= r_min; the exponent always runs (ex2(-inf) = 0)
           const int r = cc * 32 + e;
-          const float x = __uint_as_float(sv[e]) * p.scale_log2 - lse_b[r];
+          const float x = __uint_as_float(sv[e]) * p.scale_log2 - lv[e];
           P[r] = ex2(r >= r_min ? x : -INFINITY);
         }
 #pragma unroll
@@ -387,13 +399,19 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       for (int cc = 0; cc < 4; ++cc) {
         uint32_t dv[32];
         tmem_ld32(tmem + lane_base + C::TM_DPT + cc * 32, dv);
+        float dlv[32];
+#pragma unroll
+        for (int v = 0; v < 8; ++v) {
+          const float4 t4 = reinterpret_cast<const float4*>(dl_b + cc * 32)[v];
+          dlv[4 * v] = t4.x; dlv[4 * v + 1] = t4.y; dlv[4 * v + 2] = t4.z; dlv[4 * v + 3] = t4.w;
+        }
         tmem_wait_ld();
         uint32_t dk[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
           const int r = cc * 32 + 2 * e;
-          const float d0 = P[r] * (__uint_as_float(dv[2 * e]) - dl_b[r]);
-          const float d1 = P[r + 1] * (__uint_as_float(dv[2 * e + 1]) - dl_b[r + 1]);
+          const float d0 = P[r] * (__uint_as_float(dv[2 * e]) - dlv[2 * e]);
+          const float d1 = P[r + 1] * (__uint_as_float(dv[2 * e + 1]) - dlv[2 * e + 1]);
           dk[e] = pack_bf16x2(d0, d1);
         }
         tmem_st16(tmem + lane_base + C::TM_DPT + cc * 16, dk);
