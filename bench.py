@@ -87,13 +87,28 @@ def barrier(world):
 
 
 def max_over_ranks(x, world):
+    """The max of x over all ranks (the step time a job is held to)."""
     if world == 1:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def whole_job_tflops(flops_per_rank, ms_max, world):
+    """Weak scaling: every rank processes its own problem of flops_per_rank;
+    the job's throughput is all ranks' work over the slowest rank's time."""
+    return world * flops_per_rank / (ms_max * 1e-3) / 1e12
+
+
+def rank_workload(rank):
+    """The decode workload of one rank: same shapes, its own seed."""
+    import pbsa_inputs as PI
+    w = PI.WORKLOADS["decode"]
+    return PI.variant(w, seed=w.seed + 1000 * rank) if rank else w
 
 
 # ----------------------------------------------------------------- clocks
@@ -151,9 +166,7 @@ class DecodeRunner:
         import pbsa_inputs as PI
         from block_sparse_attention_39_b200.engine import PbsaLayer
         self.torch = torch
-        w = PI.WORKLOADS["decode"]
-        if seed_offset:
-            w = PI.variant(w, seed=w.seed + 1000 * seed_offset)
+        w = rank_workload(seed_offset)
         self.w = w
         snap = PI.snapshot(w)
         self.snap = snap
@@ -577,7 +590,7 @@ def main():
     ms_attn = float(per[:, 1].mean())
     ms_step_max = max_over_ranks(ms_step, world)
     flops = runner.flops()
-    value = world * flops / (ms_step_max * 1e-3) / 1e12
+    value = whole_job_tflops(flops, ms_step_max, world)
     attn_tflops = flops / (ms_attn * 1e-3) / 1e12
     peak = pk["bf16_tflops"]
     b_score, b_upd = runner.hbm_bytes()
@@ -622,7 +635,7 @@ def main():
     if not args.no_e2e:
         e2e_ms, h2d, d2h = runner.e2e(steps=min(args.steps, 50), warmup=5)
         e2e_ms = max_over_ranks(e2e_ms, world)
-        line["e2e"] = {"value": round(world * flops / (e2e_ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+        line["e2e"] = {"value": round(whole_job_tflops(flops, e2e_ms, world), 3), "unit": "TFLOP/s",
                        "ms_per_step": round(e2e_ms, 4), "h2d_bytes_per_step": h2d,
                        "d2h_bytes_per_step": d2h}
     if world == 1 and not args.no_extras:
