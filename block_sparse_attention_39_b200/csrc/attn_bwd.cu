@@ -149,9 +149,12 @@ __global__ void __launch_bounds__(256) bwd_rev_kernel(BwdParams p) {
 // The MMA warp issues dV_i, S^T_{i+1}, dK_i, dP^T_{i+1} in that order: the
 // tensor cores compute the next query block's S^T while the softmax warps
 // form dS^T_i, and every reuse of a TMEM region is safe because tcgen05 MMAs
-// issued by one thread run in order.  Thread c of the four softmax warps owns
-// key row c (TMEM lane c) and keeps its 128 probabilities in registers between
-// the P^T and dS^T passes.
+// issued by one thread run in order.  Eight softmax warps: warps w and w + 4
+// own key rows 32(w % 4) .. +31 (their TMEM lanes) and take query columns
+// [0, 64) and [64, 128) respectively, keeping their 64 probabilities in
+// registers between the P^T and dS^T passes.  Each warp writes its bf16 pairs
+// over columns it has already read: the pairs of query columns 16k .. 16k + 15
+// (MMA k-step k) sit at TMEM column 64 (k / 4) + 8 (k % 4) of the region.
 template <int D>
 struct DkdvCfg {
   static constexpr int KB = D / 64;
@@ -173,8 +176,16 @@ struct DkdvCfg {
   static constexpr int TM_COLS = 512;
 };
 
+constexpr int kBwdThreads = 320;   // 8 softmax warps, producer, MMA issuer
+constexpr int kBwdProducer = 8, kBwdMma = 9;
+
+// TMEM column of the bf16 A operand for MMA k-step k (16 rows of K each)
+__device__ __forceinline__ uint32_t a_col(int k) {
+  return static_cast<uint32_t>((k >> 2) * 64 + (k & 3) * 8);
+}
+
 template <int D>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(kBwdThreads, 1)
 bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmDO,
                 const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                 BwdParams p) {
@@ -210,13 +221,13 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     }
     mbar_init(BAR(C::B_SF), 1);
     mbar_init(BAR(C::B_DPF), 1);
-    mbar_init(BAR(C::B_PF), 4);    // one arrival per softmax warp
-    mbar_init(BAR(C::B_DSF), 4);
+    mbar_init(BAR(C::B_PF), 8);    // one arrival per softmax warp
+    mbar_init(BAR(C::B_DSF), 8);
     mbar_init(BAR(C::B_MMA), 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 4) {
+  if (warp == kBwdProducer) {
     tmem_alloc(smem_u32(tmem_holder), C::TM_COLS);
     tmem_relinquish();
   }
@@ -225,7 +236,7 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
 
-  if (warp == 4) {
+  if (warp == kBwdProducer) {
     // ---------------------------------------------------------- producer
     // K_j, V_j once; per query block: its LSE and Delta staged by the 32
     // lanes, then Q_i and dO_i by TMA into stage i & 1.
@@ -279,7 +290,7 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       }
     }
     __syncwarp();
-  } else if (warp == 5) {
+  } else if (warp == kBwdMma) {
     // ---------------------------------------------------------- MMA issuer
     if (lane == 0 && n > 0) {
       constexpr uint32_t id_kk = idesc_bf16_f32(128, 128, false, false);  // K-major x K-major
@@ -316,7 +327,7 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         tc_fence_after();
 #pragma unroll
         for (int k = 0; k < 128 / 16; ++k)        // dV += P^T dO_it
-          mma_ts(tmem + C::TM_DV, tmem + C::TM_ST + k * 8,
+          mma_ts(tmem + C::TM_DV, tmem + C::TM_ST + a_col(k),
                  smem_desc_sw128(sDO + s * C::TILE + k * 2048, C::BOX, 1024), id_kmn,
                  (it > 0 || k > 0) ? 1u : 0u);
         if (it + 1 < n && !issue_st(it + 1)) break;
@@ -324,7 +335,7 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         tc_fence_after();
 #pragma unroll
         for (int k = 0; k < 128 / 16; ++k)        // dK += dS^T Q_it
-          mma_ts(tmem + C::TM_DK, tmem + C::TM_DPT + k * 8,
+          mma_ts(tmem + C::TM_DK, tmem + C::TM_DPT + a_col(k),
                  smem_desc_sw128(sQ + s * C::TILE + k * 2048, C::BOX, 1024), id_kmn,
                  (it > 0 || k > 0) ? 1u : 0u);
         mma_commit(BAR(C::B_QE + s));
@@ -336,8 +347,10 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     __syncwarp();
   } else {
     // ---------------------------------------------------------- softmax rows
-    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
-    const int c = tid;                      // key row of the tile
+    const int q4 = warp & 3, hh = warp >> 2;  // lane quarter, half of the query columns
+    const uint32_t lane_base = static_cast<uint32_t>(q4 * 32) << 16;
+    const int c = q4 * 32 + lane;           // key row of the tile
+    const int col0 = hh * 64;               // this warp's query columns [col0, col0 + 64)
     const bool row_ok = c < klen;
     bool ok = true;
     const bool tok = p.mask == PBSA_MASK_TOKEN;
@@ -361,16 +374,16 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       const int qpos0 = p.q_pos0 + qrow0;
       // first visible query column of this key row (rows past qlen have LSE = +inf)
       const int r_min = !row_ok ? 1 << 20 : (tok ? max(0, kpos0 + c - qpos0) : 0);
-      float P[128];
+      float P[64];
 #pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
+      for (int cc = 0; cc < 2; ++cc) {
         uint32_t sv[32];
-        tmem_ld32(tmem + lane_base + C::TM_ST + cc * 32, sv);
+        tmem_ld32(tmem + lane_base + C::TM_ST + col0 + cc * 32, sv);
         // the 32 LSE values of this chunk: eight 128-bit broadcast reads
         float lv[32];
 #pragma unroll
         for (int v = 0; v < 8; ++v) {
-          const float4 t4 = reinterpret_cast<const float4*>(lse_b + cc * 32)[v];
+          const float4 t4 = reinterpret_cast<const float4*>(lse_b + col0 + cc * 32)[v];
           lv[4 * v] = t4.x; lv[4 * v + 1] = t4.y; lv[4 * v + 2] = t4.z; lv[4 * v + 3] = t4.w;
         }
         tmem_wait_ld();
@@ -378,14 +391,14 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
 #pragma unroll
         for (int e = 0; e < 32; ++e) {
           // visible columns are r >= r_min; the exponent always runs (ex2(-inf) = 0)
-          const int r = cc * 32 + e;
+          const int r = col0 + cc * 32 + e;
           const float x = __uint_as_float(sv[e]) * p.scale_log2 - lv[e];
-          P[r] = ex2(r >= r_min ? x : -INFINITY);
+          P[cc * 32 + e] = ex2(r >= r_min ? x : -INFINITY);
         }
 #pragma unroll
         for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(P[cc * 32 + 2 * e], P[cc * 32 + 2 * e + 1]);
-        // columns [16cc, 16cc + 16) of S^T were read by this chunk or the one before
-        tmem_st16(tmem + lane_base + C::TM_ST + cc * 16, pk);
+        // columns [col0 + 16cc, col0 + 16cc + 16) of S^T: this warp's, already read
+        tmem_st16(tmem + lane_base + C::TM_ST + col0 + cc * 16, pk);
       }
       tmem_wait_st();
       tc_fence_before();
@@ -396,13 +409,13 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       if (!ok) break;
       tc_fence_after();
 #pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
+      for (int cc = 0; cc < 2; ++cc) {
         uint32_t dv[32];
-        tmem_ld32(tmem + lane_base + C::TM_DPT + cc * 32, dv);
+        tmem_ld32(tmem + lane_base + C::TM_DPT + col0 + cc * 32, dv);
         float dlv[32];
 #pragma unroll
         for (int v = 0; v < 8; ++v) {
-          const float4 t4 = reinterpret_cast<const float4*>(dl_b + cc * 32)[v];
+          const float4 t4 = reinterpret_cast<const float4*>(dl_b + col0 + cc * 32)[v];
           dlv[4 * v] = t4.x; dlv[4 * v + 1] = t4.y; dlv[4 * v + 2] = t4.z; dlv[4 * v + 3] = t4.w;
         }
         tmem_wait_ld();
@@ -414,7 +427,7 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           const float d1 = P[r + 1] * (__uint_as_float(dv[2 * e + 1]) - dlv[2 * e + 1]);
           dk[e] = pack_bf16x2(d0, d1);
         }
-        tmem_st16(tmem + lane_base + C::TM_DPT + cc * 16, dk);
+        tmem_st16(tmem + lane_base + C::TM_DPT + col0 + cc * 16, dk);
       }
       tmem_wait_st();
       tc_fence_before();
@@ -431,8 +444,9 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       const bool store = c < p.bs;
       float* dvrow = p.dv + ((static_cast<long>(bh) * p.NB + j) * p.bs + c) * D;
       float* dkrow = p.dk + ((static_cast<long>(bh) * p.NB + j) * p.bs + c) * D;
+      // warps w and w + 4 store halves [0, D/2) and [D/2, D) of the row
 #pragma unroll 1
-      for (int cc = 0; cc < D / 32; ++cc) {
+      for (int cc = hh * (D / 64); cc < (hh + 1) * (D / 64); ++cc) {
         uint32_t a[32], b[32];
         if (n > 0) {
           tmem_ld32(tmem + lane_base + C::TM_DV + cc * 32, a);
@@ -458,7 +472,7 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 4) {
+  if (warp == kBwdProducer) {
     tc_fence_after();
     tmem_dealloc(tmem, C::TM_COLS);
   }
@@ -497,7 +511,7 @@ struct DqCfg {
 };
 
 template <int D, int NK, int NV>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(kBwdThreads, 1)
 bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmDO,
               const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
               BwdParams p) {
@@ -536,12 +550,12 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     mbar_init(BAR(C::B_SF), 1);
     mbar_init(BAR(C::B_SF + 1), 1);
     mbar_init(BAR(C::B_DPF), 1);
-    mbar_init(BAR(C::B_DSF), 4);    // one arrival per softmax warp
+    mbar_init(BAR(C::B_DSF), 8);    // one arrival per softmax warp
     mbar_init(BAR(C::B_MMA), 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 4) {
+  if (warp == kBwdProducer) {
     tmem_alloc(smem_u32(tmem_holder), C::TM_COLS);
     tmem_relinquish();
   }
@@ -561,7 +575,7 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     return id;
   };
 
-  if (warp == 4) {
+  if (warp == kBwdProducer) {
     // ---------------------------------------------------------- producer
     if (lane == 0 && n > 0) {
       const int q_row = bh * p.Tq + qrow0;
@@ -600,7 +614,7 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         mbar_drain(BAR(C::B_VF + jj % NV), (jj / NV) & 1, p.status, p.limit_ns);
     }
     __syncwarp();
-  } else if (warp == 5) {
+  } else if (warp == kBwdMma) {
     // ---------------------------------------------------------- MMA issuer
     if (lane == 0 && n > 0) {
       constexpr uint32_t id_kk = idesc_bf16_f32(128, 128, false, false);
@@ -644,7 +658,7 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         const uint32_t ds_tm = tmem + ((jj & 1) ? C::TM_S1 : C::TM_S0);
 #pragma unroll
         for (int k = 0; k < 128 / 16; ++k)        // dQ += dS_jj K_jj
-          mma_ts(tmem + C::TM_DQ, ds_tm + k * 8,
+          mma_ts(tmem + C::TM_DQ, ds_tm + a_col(k),
                  smem_desc_sw128(sK + ks * C::TILE + k * 2048, C::BOX, 1024), id_kmn,
                  (jj > 0 || k > 0) ? 1u : 0u);
         mma_commit(BAR(C::B_KE + ks));
@@ -659,8 +673,10 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     __syncwarp();
   } else {
     // ---------------------------------------------------------- softmax rows
-    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
-    const int r = tid;
+    const int q4 = warp & 3, hh = warp >> 2;  // lane quarter, half of the key columns
+    const uint32_t lane_base = static_cast<uint32_t>(q4 * 32) << 16;
+    const int r = q4 * 32 + lane;           // query row of the tile
+    const int col0 = hh * 64;               // this warp's key columns [col0, col0 + 64)
     const bool row_ok = r < qlen;
     float l2 = INFINITY, dl = 0.f;
     if (row_ok) {
@@ -694,18 +710,18 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       const uint32_t s_tm = tmem + lane_base + ((jj & 1) ? C::TM_S1 : C::TM_S0);
       int c_lim = row_ok ? len : 0;
       if (p.mask == PBSA_MASK_TOKEN) c_lim = min(c_lim, max(0, qpos - kpos0 + 1));
-      float P[128];
+      float P[64];
 #pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
+      for (int cc = 0; cc < 2; ++cc) {
         uint32_t sv[32];
-        tmem_ld32(s_tm + cc * 32, sv);
+        tmem_ld32(s_tm + col0 + cc * 32, sv);
         tmem_wait_ld();
 #pragma unroll
         for (int e = 0; e < 32; ++e) {
           // visible columns are col < c_lim; the exponent always runs (ex2(-inf) = 0)
-          const int col = cc * 32 + e;
+          const int col = col0 + cc * 32 + e;
           const float x = __uint_as_float(sv[e]) * p.scale_log2 - l2;
-          P[col] = ex2(col < c_lim ? x : -INFINITY);
+          P[cc * 32 + e] = ex2(col < c_lim ? x : -INFINITY);
         }
       }
       ok = mbar_wait(BAR(C::B_DPF), jj & 1, abort_flag, p.status, p.limit_ns);
@@ -713,9 +729,9 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       if (!ok) break;
       tc_fence_after();
 #pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
+      for (int cc = 0; cc < 2; ++cc) {
         uint32_t dv[32];
-        tmem_ld32(tmem + lane_base + C::TM_DP + cc * 32, dv);
+        tmem_ld32(tmem + lane_base + C::TM_DP + col0 + cc * 32, dv);
         tmem_wait_ld();
         uint32_t pk[16];
 #pragma unroll
@@ -724,8 +740,8 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
           pk[e] = pack_bf16x2(P[col] * (__uint_as_float(dv[2 * e]) - dl),
                               P[col + 1] * (__uint_as_float(dv[2 * e + 1]) - dl));
         }
-        // every column of S_jj was read above
-        tmem_st16(s_tm + cc * 16, pk);
+        // columns [col0, col0 + 64) of S_jj are this warp's and were read above
+        tmem_st16(s_tm + col0 + cc * 16, pk);
       }
       tmem_wait_st();
       tc_fence_before();
@@ -739,8 +755,9 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     if (ok) {
       tc_fence_after();
       float* dqrow = p.dq + (static_cast<long>(bh) * p.Tq + qrow0 + r) * D;
+      // warps w and w + 4 store halves [0, D/2) and [D/2, D) of the row
 #pragma unroll 1
-      for (int cc = 0; cc < D / 32; ++cc) {
+      for (int cc = hh * (D / 64); cc < (hh + 1) * (D / 64); ++cc) {
         uint32_t a[32];
         if (n > 0) {
           tmem_ld32(tmem + lane_base + C::TM_DQ + cc * 32, a);
@@ -761,7 +778,7 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 4) {
+  if (warp == kBwdProducer) {
     tc_fence_after();
     tmem_dealloc(tmem, C::TM_COLS);
   }
@@ -814,7 +831,7 @@ int launch_bwd(const pbsa_dims* d, BwdParams& p, const CUtensorMap& mq, const CU
   {
     auto kern = bwd_dkdv_kernel<D>;
     opt_in_smem<bwd_dkdv_kernel<D>>();
-    if (launch(kern, dim3(static_cast<unsigned>(BH) * p.NB), dim3(192), DkdvCfg<D>::SMEM, s, mq,
+    if (launch(kern, dim3(static_cast<unsigned>(BH) * p.NB), dim3(kBwdThreads), DkdvCfg<D>::SMEM, s, mq,
                mdo, mk, mv, p) != cudaSuccess)
       PBSA_CHECK_LAUNCH("bwd_dkdv_kernel");
   }
@@ -824,7 +841,7 @@ int launch_bwd(const pbsa_dims* d, BwdParams& p, const CUtensorMap& mq, const CU
     opt_in_smem<bwd_dq_kernel<D, NK, NV>>();
     const size_t smem = DqCfg<D, NK, NV>::SMEM;
     static_assert(DqCfg<128, 3, 2>::SMEM <= 227 * 1024, "dQ tiles exceed shared memory");
-    if (launch(kern, dim3(static_cast<unsigned>(BH) * p.nQB), dim3(192), smem, s, mq, mdo, mk, mv,
+    if (launch(kern, dim3(static_cast<unsigned>(BH) * p.nQB), dim3(kBwdThreads), smem, s, mq, mdo, mk, mv,
                p) != cudaSuccess)
       PBSA_CHECK_LAUNCH("bwd_dq_kernel");
   }
