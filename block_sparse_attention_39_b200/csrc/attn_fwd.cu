@@ -322,13 +322,14 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       const int kpos0 = s_pos[j];
       // masking only for partial blocks and blocks that reach past the first query
       const bool tok = p.mask == PBSA_MASK_TOKEN && kpos0 + BS - 1 > qpos_first;
-      if (len < BS || tok) {
+      {
+        // visible keys are c < lim: one bound per row and a select per element,
+        // on every block.  A separate branch taken only by partial blocks cost
+        // about 8k cycles each time it ran (measured with clock stamps).
+        int lim = len;
+        if (tok) lim = min(lim, max(0, qpos - kpos0 + 1));
 #pragma unroll
-        for (int c = 0; c < BS; ++c) {
-          bool vis = c < len;
-          if (tok) vis = vis && (kpos0 + c <= qpos);
-          if (!vis) sr[c] = __float_as_uint(-INFINITY);
-        }
+        for (int c = 0; c < BS; ++c) sr[c] = c < lim ? sr[c] : __float_as_uint(-INFINITY);
       }
       float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
