@@ -79,7 +79,8 @@ struct FwdCfg {
   static constexpr int B_PF = B_SF + 2;                  // + stream (2)
   static constexpr int B_OD = B_PF + 2;                  // + stream (2)
   static constexpr int B_ST = B_OD + 2;                  // stream 1's statistics written
-  static constexpr int B_MMA = B_ST + 1;
+  static constexpr int B_ST2 = B_ST + 1;                 // merge weights written back
+  static constexpr int B_MMA = B_ST2 + 1;
   static constexpr int NBAR = B_MMA + 1;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int OFF_IDS = OFF_MISC + 16;
@@ -160,9 +161,18 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       mbar_init(BAR(C::B_OD + h), 1);
     }
     mbar_init(BAR(C::B_ST), 128);
+    mbar_init(BAR(C::B_ST2), 128);
     mbar_init(BAR(C::B_MMA), 1);
     *abort_flag = 0;
     fence_mbar_init();
+    // Q does not depend on the list: its load overlaps the list staging below
+    if (n > 0) {
+      prefetch_tmap(&tmQ);
+      mbar_expect_tx(BAR(C::B_Q), C::Q_BYTES);
+#pragma unroll
+      for (int kb = 0; kb < C::KB; ++kb)
+        tma_load_2d(sQ + kb * C::BOX_Q, &tmQ, BAR(C::B_Q), kb * 64, bh * p.Tq + qrow0);
+    }
   }
   const int32_t* row_ids = p.idx + (static_cast<long>(bh) * p.nQB + qi) * p.Amax;
   for (int e = tid; e < n; e += blockDim.x) {
@@ -194,13 +204,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     // K_j and V_j in list order.  V_j waits for PV_{j-NSV}, which always
     // completes before K_{j+1} is needed (QK_{j+1} is issued after PV_{j-1}).
     if (lane == 0 && n > 0) {
-      prefetch_tmap(&tmQ);
       prefetch_tmap(&tmK);
       prefetch_tmap(&tmV);
-      const int q_row = bh * p.Tq + qrow0;
-      mbar_expect_tx(BAR(C::B_Q), C::Q_BYTES);
-#pragma unroll
-      for (int kb = 0; kb < C::KB; ++kb) tma_load_2d(sQ + kb * C::BOX_Q, &tmQ, BAR(C::B_Q), kb * 64, q_row);
       const bool skip_v0 = (p.debug & 1) != 0;
       int k_issued = 0, v_issued = 0;
       for (int j = 0; j < n; ++j) {
@@ -418,57 +423,75 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       ok = mbar_wait(BAR(C::B_OD + h), (n_h - 1) & 1, abort_flag, p.status, p.limit_ns);
       ok = __all_sync(0xffffffffu, ok);
     }
+    // Merge the two streams: stream 1 hands its (m, l) to stream 0, which
+    // writes back the weights of O0 and O1; then each stream normalises and
+    // stores half of the row's columns (and stream 0 the LSE).
+    const int n1 = n / 2;
+    float w0 = 0.f, w1 = 0.f, m = -INFINITY, lt = 0.f;
     if (h == 1) {
-      // hand this stream's statistics to stream 0, which writes the output
       st_m1[row] = m_use;
       st_l1[row] = l;
       tc_fence_before();
       mbar_arrive(BAR(C::B_ST));
+      bool ok2 = mbar_wait(BAR(C::B_ST2), 0, abort_flag, p.status, p.limit_ns);
+      ok = __all_sync(0xffffffffu, ok && ok2);
+      if (ok) {
+        w0 = st_m1[row];
+        w1 = st_l1[row];
+      }
     } else {
       bool ok1 = mbar_wait(BAR(C::B_ST), 0, abort_flag, p.status, p.limit_ns);
       ok = __all_sync(0xffffffffu, ok && ok1);
       if (ok) {
-        tc_fence_after();
-        const int n1 = n / 2;
         const float m1 = st_m1[row], l1 = st_l1[row];
-        const float m = fmaxf(m_use, m1);
+        m = fmaxf(m_use, m1);
         const float a0 = (m_use == -INFINITY) ? 0.f : ex2(m_use - m);
         const float a1 = (m1 == -INFINITY || n1 == 0) ? 0.f : ex2(m1 - m);
-        const float lt = a0 * l + a1 * l1;
+        lt = a0 * l + a1 * l1;
         const float inv = lt > 0.f ? 1.f / lt : 0.f;
-        const float w0 = a0 * inv, w1 = a1 * inv;
-        const bool valid = row < qlen;
-        __nv_bfloat16* orow = p.o + (static_cast<long>(bh) * p.Tq + qrow0 + row) * D;
+        w0 = a0 * inv;
+        w1 = a1 * inv;
+        st_m1[row] = w0;
+        st_l1[row] = w1;
+      }
+      tc_fence_before();
+      mbar_arrive(BAR(C::B_ST2));
+    }
+    if (ok) {
+      tc_fence_after();
+      const bool valid = row < qlen;
+      __nv_bfloat16* orow = p.o + (static_cast<long>(bh) * p.Tq + qrow0 + row) * D;
+      constexpr int HALF = D / 64;             // 32-column chunks per stream
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t o0[32], o1[32];
-          if (n > 0) tmem_ld32(tmem + lane_base + C::TM_O0 + c * 32, o0);
-          if (n1 > 0) tmem_ld32(tmem + lane_base + C::TM_O1 + c * 32, o1);
-          tmem_wait_ld();
-          float v[32];
+      for (int cc = 0; cc < HALF; ++cc) {
+        const int c = h * HALF + cc;
+        uint32_t o0[32], o1[32];
+        if (n > 0) tmem_ld32(tmem + lane_base + C::TM_O0 + c * 32, o0);
+        if (n1 > 0) tmem_ld32(tmem + lane_base + C::TM_O1 + c * 32, o1);
+        tmem_wait_ld();
+        float v[32];
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            float x = n > 0 ? __uint_as_float(o0[e]) * w0 : 0.f;
-            if (n1 > 0) x = fmaf(__uint_as_float(o1[e]), w1, x);
-            v[e] = x;
-          }
-          if (valid) {
-            uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+        for (int e = 0; e < 32; ++e) {
+          float x = n > 0 ? __uint_as_float(o0[e]) * w0 : 0.f;
+          if (n1 > 0) x = fmaf(__uint_as_float(o1[e]), w1, x);
+          v[e] = x;
+        }
+        if (valid) {
+          uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
 #pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4) {
-              uint4 u;
-              u.x = pack_bf16x2(v[8 * q4 + 0], v[8 * q4 + 1]);
-              u.y = pack_bf16x2(v[8 * q4 + 2], v[8 * q4 + 3]);
-              u.z = pack_bf16x2(v[8 * q4 + 4], v[8 * q4 + 5]);
-              u.w = pack_bf16x2(v[8 * q4 + 6], v[8 * q4 + 7]);
-              dst[q4] = u;
-            }
+          for (int q4 = 0; q4 < 4; ++q4) {
+            uint4 u;
+            u.x = pack_bf16x2(v[8 * q4 + 0], v[8 * q4 + 1]);
+            u.y = pack_bf16x2(v[8 * q4 + 2], v[8 * q4 + 3]);
+            u.z = pack_bf16x2(v[8 * q4 + 4], v[8 * q4 + 5]);
+            u.w = pack_bf16x2(v[8 * q4 + 6], v[8 * q4 + 7]);
+            dst[q4] = u;
           }
         }
-        if (valid)
-          p.lse[static_cast<long>(bh) * p.Tq + qrow0 + row] =
-              lt > 0.f ? (m + __log2f(lt)) * 0.69314718055994531f : -INFINITY;
       }
+      if (h == 0 && valid)
+        p.lse[static_cast<long>(bh) * p.Tq + qrow0 + row] =
+            lt > 0.f ? (m + __log2f(lt)) * 0.69314718055994531f : -INFINITY;
     }
   }
 
