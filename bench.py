@@ -38,6 +38,22 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+# DRAM bytes (read + write) of one attn_fwd launch on the decode step, from an
+# ncu capture (profiles/decode_step_kernels_full.md), keyed by a hash of the
+# kernel's sources: a changed kernel reports null until it is captured again.
+ATTN_TRAFFIC_SOURCES = ["attn_fwd.cu", "tc_sm100.cuh", "common.cuh", "launch.h", "tmap.h"]
+ATTN_TRAFFIC = {"659c99594586ecd3d63a16f49864e45c0e937d163719a42bc00377e713b5cf36": 97268736}
+
+
+def attn_traffic():
+    import hashlib
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "block_sparse_attention_39_b200", "csrc")
+    for f in ATTN_TRAFFIC_SOURCES:
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(fh.read())
+    return ATTN_TRAFFIC.get(h.hexdigest())
 L2_FLUSH_BYTES = 256 << 20
 
 
@@ -47,7 +63,9 @@ def parse():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="pbsa", choices=["pbsa", "reference"])
-    ap.add_argument("--workload", default="decode", choices=["decode"])
+    ap.add_argument("--workload", default="decode", choices=["decode", "train"],
+                    help="decode: the decode step (default); train: forward + backward of "
+                         "the trainable shape on its P32 + top-16 lists")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-extras", action="store_true",
@@ -535,6 +553,8 @@ def main():
     args = parse()
     if args.impl == "reference":
         return run_reference(args)
+    if args.workload == "train":
+        return run_train(args)
     import torch
     rank, world, local = init_dist(args.gpus)
     pk, pk_kind = peaks()
@@ -625,7 +645,8 @@ def main():
         "attended_gflop_per_step": round(flops / 1e9, 3),
         "roofline": {"kernel": "attn_fwd_kernel (D=128, bs=128)", "bound": "tensor",
                      "achieved": round(attn_tflops, 2), "peak": peak, "unit": "TFLOP/s",
-                     "frac": round(attn_tflops / peak, 4), "traffic": None,
+                     "frac": round(attn_tflops / peak, 4), "traffic": attn_traffic(),
+                     "traffic_unit": "bytes per launch (ncu dram read + write)",
                      "peak_kind": f"bf16_tflops burst, {pk_kind}"},
         "hbm": hbm,
         "gpu_launches": runner.launches_per_step * args.steps,
@@ -650,6 +671,64 @@ def main():
                                 "cores": cores_used(), "kind": "oracle", "sample": desc,
                                 "seconds": round(dt, 2)}
     if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def run_train(args):
+    """Forward + backward of the trainable shape (B2 H12 D128, 32 760 tokens) on
+    the lists the library builds (persistent top-32 + local top-16).  One step
+    is one forward and one backward; the metric counts 4 (forward) + 10
+    (backward) x len_q x len_k x D FLOP per attended pair."""
+    import torch
+    import pbsa_inputs as PI
+    from block_sparse_attention_39_b200.engine import PbsaTrain
+    rank, world, local = init_dist(args.gpus)
+    w = PI.WORKLOADS["train"]
+    T = PbsaTrain(w)
+    g = torch.Generator(device="cuda").manual_seed(w.seed + 1000 * rank)
+    for t in (T.q, T.dO, T.kpool, T.vpool):
+        t.copy_(torch.randn(t.shape, generator=g, device="cuda").bfloat16())
+    T.set_meta()
+    T.lists()
+    torch.cuda.synchronize()
+    lens = np.array([n for c in range(w.n_chunks) for n in w.chunk_block_lens()], dtype=np.int64)
+    ffl = _pair_flops(T.idx.cpu().numpy(), T.cnt.cpu().numpy(), T.blk_len.cpu().numpy(), lens,
+                      w.D, 4)
+    flops = ffl * (4 + 10) // 4
+    for _ in range(args.warmup):
+        T.fwd()
+        T.bwd()
+    torch.cuda.synchronize()
+    s = torch.cuda.current_stream()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    barrier(world)
+    for e in ev:
+        e[0].record(s)
+        T.fwd()
+        e[1].record(s)
+        T.bwd()
+        e[2].record(s)
+    torch.cuda.synchronize()
+    barrier(world)
+    ms_f = float(np.mean([a.elapsed_time(b) for a, b, _ in ev]))
+    ms_b = float(np.mean([b.elapsed_time(c) for _, b, c in ev]))
+    ms = max_over_ranks(ms_f + ms_b, world)
+    if rank == 0:
+        line = {"metric": "PBSA fwd+bwd effective TFLOP/s (trainable shape)",
+                "value": round(whole_job_tflops(flops, ms, world), 3), "unit": "TFLOP/s",
+                "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1))",
+                "config": {"workload": f"trainable shape B{w.B} H{w.H} D{w.D}, {T.T} tokens, "
+                                       f"lists P{w.P} + top-{w.k}", "parallelism": "replicas"},
+                "fwd_ms": round(ms_f, 4), "bwd_ms": round(ms_b, 4),
+                "fwd_tflops": round(ffl / ms_f / 1e9, 1),
+                "bwd_tflops": round(2.5 * ffl / ms_b / 1e9, 1),
+                "gpu_launches": args.steps * 5}
         print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist
