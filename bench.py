@@ -493,6 +493,72 @@ def bench_rollouts(torch, timed_steps=6):
     return out
 
 
+def bench_hbm_at_scale(torch, flush, pk, reps=5):
+    """The HBM-bound calls on bandwidth-sized work, beside the latency-bound
+    decode step: score_blocks pooling and scoring the whole trainable shape
+    (every query and key block of 32 760 tokens, B2 H12), and update_memory
+    filling 128 slots per head from 111 candidate blocks (B2 H12)."""
+    import pbsa_inputs as PI
+    from block_sparse_attention_39_b200 import pbsa as K
+    from block_sparse_attention_39_b200.engine import PbsaLayer, PbsaTrain
+    out = {}
+    w = PI.WORKLOADS["train"]
+    T = PbsaTrain(w)
+    g = torch.Generator(device="cuda").manual_seed(5)
+    for t in (T.q, T.kpool):
+        t.copy_(torch.randn(t.shape, generator=g, device="cuda").bfloat16())
+    T.set_meta()
+    fn = lambda: K.score_blocks(T.d, T.q, T.T, T.kpool, T.NB, T.blk_len, T.all_ids, T.NB,
+                                T.q_bar, T.k_bar, T.scores, T.mem)
+    fn()
+    # inputs (415 MB) exceed the 126 MB L2, so no flush between repetitions: a
+    # flush leaves dirty lines whose write-back would land in the timed call
+    ms = _timed(torch, fn, reps, None)
+    BH = w.B * w.H
+    byt = (BH * T.T * w.D * 2 * 2                    # Q and every key row read
+           + BH * (T.nQB + T.NB) * w.D * 4           # q_bar, k_bar written
+           + BH * T.nQB * T.NB * 4 + BH * T.G * T.NB * 4)   # S and m written
+    out["score_blocks, trainable shape"] = {
+        "bytes": byt, "ms": round(ms, 4), "gbs": round(byt / ms / 1e6, 1),
+        "frac": round(byt / ms / 1e6 / pk["hbm_gbs"], 4)}
+    del T
+    torch.cuda.empty_cache()
+    wv = PI.variant(PI.WORKLOADS["decode"], B=2, P=128)
+    L = PbsaLayer(wv)
+    for t in (L.kpool, L.vpool):
+        t.copy_(torch.randn(t.shape, generator=g, device="cuda").bfloat16())
+    for c in range(wv.n_chunks):
+        L.set_chunk_meta(c)
+    L.score(wv.n_chunks - 1, pool_ids=L.ids(("all",), [p for c in range(wv.n_chunks)
+                                                       for p in wv.chunk_phys_ids(c)]))
+    ci, cs = L.candidates(wv.n_chunks - 1)
+
+    L.reset_memory()
+    L.update(ci, cs)
+    torch.cuda.synchronize()
+    kept = int((L.slot_src >= 0).sum().item())
+    s = torch.cuda.current_stream()
+    tl = []
+    for _ in range(reps):                # the update call alone (memory reset before; the
+        L.reset_memory()                 # 352 MB it moves exceed L2, so no flush)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(s)
+        L.update(ci, cs)
+        b.record(s)
+        tl.append((a, b))
+    torch.cuda.synchronize()
+    ms = float(np.mean([a.elapsed_time(b) for a, b in tl]))
+    byt = kept * (wv.bs * wv.D * 2 * 2 * 2 + wv.D * 4 * 2)
+    out["update_memory, 128 slots from 111 candidates, B2 H12"] = {
+        "bytes": byt, "ms": round(ms, 4), "gbs": round(byt / ms / 1e6, 1),
+        "frac": round(byt / ms / 1e6 / pk["hbm_gbs"], 4)}
+    del L
+    torch.cuda.empty_cache()
+    out["peak_gbs"] = pk["hbm_gbs"]
+    out["l2"] = "not flushed: every input is larger than the 126 MB L2"
+    return out
+
+
 # ----------------------------------------------------------------- CPU oracle
 def cpu_oracle_sample(w, snap, n_heads=2, n_qblocks=None):
     """Time the oracle on a bounded sample: the full score/update/select on the
@@ -664,6 +730,7 @@ def main():
                                                                                  runner.flush_buf)}
         extras["train"] = bench_train(torch, runner.flush_buf)
         extras["rollouts"] = bench_rollouts(torch)
+        extras["hbm_at_scale"] = bench_hbm_at_scale(torch, runner.flush_buf, pk)
         line["extras"] = extras
     if rank == 0 and not args.no_cpu:
         fl, dt, desc = cpu_oracle_sample(w, runner.snap)
