@@ -360,6 +360,38 @@ def _timed(torch, fn, reps, flush=None):
     return float(np.mean([a.elapsed_time(b) for a, b in ts]))
 
 
+def _graph_timed(torch, fn, reps, pre=None):
+    """Mean device time (ms) of fn() captured in CUDA graphs with its timing
+    events inside the graph, so host launch overhead is not timed; pre() (if
+    given) runs in the same graph before the first event."""
+    s = torch.cuda.Stream()
+    torch.cuda.synchronize()
+    with torch.cuda.stream(s):
+        for _ in range(2):
+            if pre is not None:
+                pre()
+            fn()
+    torch.cuda.synchronize()
+    graphs = []
+    for _ in range(reps):
+        ev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(2)]
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=s):
+            if pre is not None:
+                pre()
+            ev[0].record()
+            fn()
+            ev[1].record()
+        graphs.append((g, ev))
+    with torch.cuda.stream(s):
+        for g, _ in graphs:
+            g.replay()
+    torch.cuda.synchronize()
+    ms = float(np.mean([ev[0].elapsed_time(ev[1]) for _, ev in graphs]))
+    del graphs
+    return ms
+
+
 def _pair_flops(idx, cnt, blk_len, q_lens, D, per_pair):
     total = 0
     B, H, nQB = cnt.shape
@@ -459,27 +491,38 @@ def bench_rollouts(torch, timed_steps=6):
         steps = warm + timed_steps
         def draw():
             return tuple(torch.randn(shape, generator=g, device="cuda").bfloat16() for _ in range(3))
+        # warm-up steps run eagerly; each timed step is a CUDA graph of every
+        # layer's score -> update -> select -> attend with the timing events
+        # inside it (so host launch overhead is not timed), replayed after the
+        # step's new chunk has been written
+        gs = torch.cuda.Stream()
         times = []
         for t in range(steps):
-            if t >= warm:
-                pre = [draw() for _ in layers]          # drawn before the timed region
-            s = torch.cuda.current_stream()
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            pre = [draw() for _ in layers]
             for li, L in enumerate(layers):
-                q, k, v = pre[li] if t >= warm else draw()
+                q, k, v = pre[li]
                 L.write_chunk(t, k, v)
                 L.q.copy_(q)
-                L.candidates(t)                 # id lists built before the timed region
+                L.candidates(t)                 # id lists built outside the timed region
                 L.window_ids(t)
                 L.chunk_ids(t)
-            if t >= warm:
-                torch.cuda.synchronize()
-                a.record(s)
-            for L in layers:
-                L.step(t)
-            if t >= warm:
-                b.record(s)
-                times.append((a, b))
+            if t < warm:
+                for L in layers:
+                    L.step(t)
+                continue
+            torch.cuda.synchronize()
+            ev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(2)]
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph, stream=gs):
+                ev[0].record()
+                for L in layers:
+                    L.step(t)
+                ev[1].record()
+            with torch.cuda.stream(gs):
+                graph.replay()
+            torch.cuda.synchronize()
+            times.append(tuple(ev))
+            del graph
         torch.cuda.synchronize()
         ms = float(np.mean([a.elapsed_time(b) for a, b in times]))
         kv = sum(layer_bytes(L) for L in layers)
@@ -513,7 +556,7 @@ def bench_hbm_at_scale(torch, flush, pk, reps=5):
     fn()
     # inputs (415 MB) exceed the 126 MB L2, so no flush between repetitions: a
     # flush leaves dirty lines whose write-back would land in the timed call
-    ms = _timed(torch, fn, reps, None)
+    ms = _graph_timed(torch, fn, reps)
     BH = w.B * w.H
     byt = (BH * T.T * w.D * 2 * 2                    # Q and every key row read
            + BH * (T.nQB + T.NB) * w.D * 4           # q_bar, k_bar written
@@ -537,17 +580,9 @@ def bench_hbm_at_scale(torch, flush, pk, reps=5):
     L.update(ci, cs)
     torch.cuda.synchronize()
     kept = int((L.slot_src >= 0).sum().item())
-    s = torch.cuda.current_stream()
-    tl = []
-    for _ in range(reps):                # the update call alone (memory reset before; the
-        L.reset_memory()                 # 352 MB it moves exceed L2, so no flush)
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(s)
-        L.update(ci, cs)
-        b.record(s)
-        tl.append((a, b))
-    torch.cuda.synchronize()
-    ms = float(np.mean([a.elapsed_time(b) for a, b in tl]))
+    # the update call alone, the memory reset before it in the same graph (the
+    # 352 MB it moves exceed L2, so no flush)
+    ms = _graph_timed(torch, lambda: L.update(ci, cs), reps, pre=L.reset_memory)
     byt = kept * (wv.bs * wv.D * 2 * 2 * 2 + wv.D * 4 * 2)
     out["update_memory, 128 slots from 111 candidates, B2 H12"] = {
         "bytes": byt, "ms": round(ms, 4), "gbs": round(byt / ms / 1e6, 1),
@@ -556,6 +591,7 @@ def bench_hbm_at_scale(torch, flush, pk, reps=5):
     torch.cuda.empty_cache()
     out["peak_gbs"] = pk["hbm_gbs"]
     out["l2"] = "not flushed: every input is larger than the 126 MB L2"
+    out["timed"] = "CUDA graphs with the timing events inside, device time of the call"
     return out
 
 

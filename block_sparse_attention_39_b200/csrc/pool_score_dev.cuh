@@ -241,7 +241,7 @@ __host__ __device__ inline int pool_stages(int bs) {
 }
 
 constexpr int kScoreJ = 16;     // key blocks per CTA
-constexpr int kScoreQI = 128;   // query blocks staged per pass
+constexpr int kScoreQI = 64;    // query blocks staged per pass
 constexpr int kScoreTileMax = 1024;   // query blocks whose S columns stay in shared memory
 
 struct ScoreArgs {

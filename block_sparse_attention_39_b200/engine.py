@@ -180,9 +180,11 @@ class PbsaLayer:
                      mem_ids=self.mem_ids, n_mem=self.P, mask=w.mask, q_pos0=t * w.chunk_tokens,
                      idx=self.idx, cnt=self.cnt, Amax=self.Amax)
 
-    def step(self, t, stream=None, fused=True):
+    def step(self, t, stream=None, fused=False):
         """Score -> update -> select -> attend for chunk t (its Q already in self.q,
-        its K/V already in the pool).  fused: the first three as one routing call."""
+        its K/V already in the pool).  fused: the first three as one routing call
+        (pbsa_route_step); the default is the per-call path, which is the faster
+        schedule on the decode and rollout shapes."""
         if fused:
             self.route(t, stream=stream)
         else:

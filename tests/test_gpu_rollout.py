@@ -188,8 +188,10 @@ def test_rollout1min_one_layer_evict_reseeded():
     _run_rollout(w, steps=8, attn_steps={7})
 
 
-def test_free_running_rollout_invariants():
-    # all 27 steps of the 20-second rollout on the GPU alone: budget, list
+@pytest.mark.parametrize("fused", [False, True])
+def test_free_running_rollout_invariants(fused):
+    # all 27 steps of the 20-second rollout on the GPU alone, through the
+    # per-call path and through the fused routing call: budget, list
     # structure and weights stay consistent at every step
     w = PI.WORKLOADS["rollout20s"]
     L = PbsaLayer(w)
@@ -198,7 +200,7 @@ def test_free_running_rollout_invariants():
         q, k, v = PI.chunk_tensors(w, t)
         L.write_chunk(t, torch.from_numpy(k).cuda().bfloat16(), torch.from_numpy(v).cuda().bfloat16())
         L.q.copy_(dev_storage(q, w.dtype))
-        L.step(t)
+        L.step(t, fused=fused)
         torch.cuda.synchronize()
         if w.leaving_chunk(t) is not None:
             admitted += w.nb_c

@@ -132,12 +132,12 @@ def test_route_inside_a_cuda_graph():
     torch.cuda.synchronize()
     with torch.cuda.stream(s):
         Lb.reset_memory()
-        Lb.step(t)                       # warm-up outside the capture
+        Lb.step(t, fused=True)           # warm-up outside the capture
     torch.cuda.synchronize()
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g, stream=s):
         Lb.reset_memory()
-        Lb.step(t)
+        Lb.step(t, fused=True)
     for _ in range(3):
         g.replay()
     torch.cuda.synchronize()
