@@ -215,15 +215,18 @@ class DecodeRunner:
         self.fused = False
         self.launches_per_step = 6   # pool, score, plan, apply, select, attention
 
-    def step(self, ev=None, fused=None):
+    def step(self, ev=None, fused=None, appended=False):
         """One step.  fused: the routing call (pbsa_route_step) then attention;
         otherwise the per-call path (score, update, select, attention).  `ev`
-        records an event between the calls."""
+        records an event between the calls.  appended: the chunk came in through
+        pbsa_append_chunk, so its keys are pooled already."""
         L = self.L
         if fused is None:
             fused = self.fused
-        calls = ([lambda: L.route(self.t)] if fused else
-                 [lambda: L.score(self.t), lambda: L.update(*self.cand), lambda: L.select(self.t)])
+        pids = L._no_ids if appended else None
+        calls = ([lambda: L.route(self.t, appended=appended)] if fused else
+                 [lambda: L.score(self.t, pool_ids=pids), lambda: L.update(*self.cand),
+                  lambda: L.select(self.t)])
         calls.append(lambda: L.attend(self.t))
         for k, c in enumerate(calls):
             if ev is not None:
@@ -231,6 +234,16 @@ class DecodeRunner:
             c()
         if ev is not None:
             ev[len(calls)].record()
+
+    def chunk_kv(self):
+        """The step's chunk as the [B,H,T_c,D] K and V a caller appends."""
+        torch, w = self.torch, self.w
+        ids = w.chunk_phys_ids(self.t)
+
+        def rows(pool):
+            x = pool[:, :, ids].reshape(w.B, w.H, len(ids) * w.bs, w.D)[:, :, :w.chunk_tokens]
+            return torch.from_numpy(np.ascontiguousarray(x)).to(torch.bfloat16)
+        return rows(self.snap["kpool"]), rows(self.snap["vpool"])
 
     def prologue(self):
         self.L.reset_memory()
@@ -306,23 +319,19 @@ class DecodeRunner:
 
     def e2e(self, steps, warmup):
         """Through the public API with host buffers, as a decode loop runs it: every
-        step copies its Q and new-chunk K/V from pinned host memory and reads its
-        O and LSE back.  The copies of step t+1's inputs and of step t-1's outputs
-        run on their own streams while step t computes (double-buffered device
-        staging); the time is the whole loop's device time over the steps."""
+        step copies its Q and new-chunk K/V [B,H,T_c,D] from pinned host memory,
+        appends the chunk to the cache (pbsa_append_chunk, which pools its keys),
+        runs the step and reads its O and LSE back.  The copies of step t+1's
+        inputs and of step t-1's outputs run on their own streams while step t
+        computes (double-buffered device staging); the time is the whole loop's
+        device time over the steps."""
         torch = self.torch
         L, w = self.L, self.w
-        ids = w.chunk_phys_ids(self.t)
-        p0, p1 = ids[0], ids[-1] + 1
         hq = torch.from_numpy(self.snap["q"]).to(torch.bfloat16).pin_memory()
-        hk = torch.from_numpy(np.ascontiguousarray(self.snap["kpool"][:, :, p0:p1])).to(
-            torch.bfloat16).pin_memory()
-        hv = torch.from_numpy(np.ascontiguousarray(self.snap["vpool"][:, :, p0:p1])).to(
-            torch.bfloat16).pin_memory()
+        ck, cv = self.chunk_kv()
+        hk, hv = ck.pin_memory(), cv.pin_memory()
         ho = [torch.empty(L.o.shape, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
         hl = [torch.empty(L.lse.shape, dtype=torch.float32).pin_memory() for _ in range(2)]
-        dk = L.kpool[:, :, p0:p1]
-        dv = L.vpool[:, :, p0:p1]
         q_st = [torch.empty_like(L.q) for _ in range(2)]
         k_st = [torch.empty(hk.shape, dtype=torch.bfloat16, device="cuda") for _ in range(2)]
         v_st = [torch.empty(hv.shape, dtype=torch.bfloat16, device="cuda") for _ in range(2)]
@@ -356,10 +365,9 @@ class DecodeRunner:
                 s_cmp.wait_event(ev_in[it])
                 L.reset_memory()                       # each step starts from empty memory
                 L.q.copy_(q_st[b])
-                dk.copy_(k_st[b])
-                dv.copy_(v_st[b])
+                L.append(self.t, k_st[b], v_st[b])
                 ev_used[it] = mark(s_cmp)
-                self.step()
+                self.step(appended=True)
                 if it >= 2:
                     s_cmp.wait_event(ev_out[it - 2])   # output staging b is free
                 o_st[b].copy_(L.o)
@@ -573,11 +581,19 @@ def bench_rollouts(torch, timed_steps=6):
     return out
 
 
+def append_traffic(BH, Tc, nb, bs, D):
+    """Algorithmic HBM bytes of pbsa_append_chunk (bf16): K and V rows read
+    once, their blocks (padding included) written once, the pooled keys and the
+    two metadata words of each block written."""
+    return BH * (2 * Tc * D * 2 + 2 * nb * bs * D * 2 + nb * D * 4 + nb * 8)
+
+
 def bench_hbm_at_scale(torch, flush, pk, reps=5):
     """The HBM-bound calls on bandwidth-sized work, beside the latency-bound
     decode step: score_blocks pooling and scoring the whole trainable shape
-    (every query and key block of 32 760 tokens, B2 H12), and update_memory
-    filling 128 slots per head from 111 candidate blocks (B2 H12)."""
+    (every query and key block of 32 760 tokens, B2 H12), update_memory
+    filling 128 slots per head from 111 candidate blocks (B2 H12), and
+    append_chunk placing a 32 760-token chunk (B2 H12, 805 MB moved)."""
     import pbsa_inputs as PI
     from block_sparse_attention_39_b200 import pbsa as K
     from block_sparse_attention_39_b200.engine import PbsaLayer, PbsaTrain
@@ -626,8 +642,56 @@ def bench_hbm_at_scale(torch, flush, pk, reps=5):
         "frac": round(byt / ms / 1e6 / pk["hbm_gbs"], 4)}
     del L
     torch.cuda.empty_cache()
+    # bandwidth-sized: inputs and pool (805 MB) exceed L2, no flush
+    B, H, D, bs, Tc = 2, 12, 128, 128, 32760
+    nb = -(-Tc // bs)
+    d = K.dims(B, H, D, bs, 1 / math.sqrt(D), torch.bfloat16)
+    g = torch.Generator(device="cuda").manual_seed(9)
+    kb = torch.randn(B, H, Tc, D, generator=g, device="cuda").bfloat16()
+    vb = torch.randn(B, H, Tc, D, generator=g, device="cuda").bfloat16()
+    kp = torch.empty(B, H, nb, bs, D, dtype=torch.bfloat16, device="cuda")
+    vp = torch.empty_like(kp)
+    bl = torch.empty(B, H, nb, dtype=torch.int32, device="cuda")
+    bp = torch.empty_like(bl)
+    kbar = torch.empty(B, H, nb, D, dtype=torch.float32, device="cuda")
+    ids = torch.randperm(nb, generator=torch.Generator().manual_seed(3)).int().cuda()
+    fn = lambda: K.append_chunk(d, kb, vb, Tc, 0, kp, vp, nb, ids, bl, bp, kbar)
+    ms = _graph_timed(torch, fn, reps)
+    byt = append_traffic(B * H, Tc, nb, bs, D)
+    out["append_chunk, 32 760-token chunk, B2 H12"] = {
+        "bytes": byt, "ms": round(ms, 4), "gbs": round(byt / ms / 1e6, 1),
+        "frac": round(byt / ms / 1e6 / pk["hbm_gbs"], 4)}
+    del kb, vb, kp, vp, bl, bp, kbar
+    torch.cuda.empty_cache()
     out["peak_gbs"] = pk["hbm_gbs"]
     out["l2"] = "not flushed: every input is larger than the 126 MB L2"
+    out["timed"] = "CUDA graphs with the timing events inside, device time of the call"
+    return out
+
+
+def bench_append(torch, runner, pk, reps=20):
+    """pbsa_append_chunk, the KV append with the keys' block pooling fused in,
+    on the decode step's chunk (B1 H12, 4680 tokens); after it the step's score
+    call pools only the queries.  The bandwidth-sized case is in
+    bench_hbm_at_scale."""
+    L, w, t = runner.L, runner.w, runner.t
+    flush = runner.flush_buf
+    k, v = (x.cuda() for x in runner.chunk_kv())
+
+    def entry(byt, ms):
+        return {"bytes": int(byt), "ms": round(ms, 5), "gbs": round(byt / ms / 1e6, 1),
+                "frac": round(byt / ms / 1e6 / pk["hbm_gbs"], 4)}
+    out = {}
+    # decode chunk: 29 MB of inputs fit L2, so the graph flushes it first (as the step does)
+    ms = _graph_timed(torch, lambda: L.append(t, k, v), reps, pre=flush.zero_)
+    out["append_chunk, decode chunk"] = entry(append_traffic(w.B * w.H, w.chunk_tokens, w.nb_c, w.bs,
+                                                      w.D), ms)
+    out["score_blocks, keys pooled by the append (queries only)"] = {
+        "ms": round(_graph_timed(torch, lambda: L.score(t, pool_ids=L._no_ids), reps,
+                                 pre=flush.zero_), 5)}
+    out["score_blocks, pooling the chunk's keys itself"] = {
+        "ms": round(_graph_timed(torch, lambda: L.score(t), reps, pre=flush.zero_), 5)}
+    out["peak_gbs"] = pk["hbm_gbs"]
     out["timed"] = "CUDA graphs with the timing events inside, device time of the call"
     return out
 
@@ -809,6 +873,7 @@ def main():
         extras["train"] = bench_train(torch, runner.flush_buf)
         extras["rollouts"] = bench_rollouts(torch)
         extras["hbm_at_scale"] = bench_hbm_at_scale(torch, runner.flush_buf, pk)
+        extras["append_chunk"] = bench_append(torch, runner, pk)
         line["extras"] = extras
     if rank == 0 and not args.no_cpu:
         fl, dt, desc = cpu_oracle_sample(w, runner.snap)
@@ -888,13 +953,15 @@ def run_hbm(args):
     res = bench_hbm_at_scale(torch, None, pk, reps=max(1, args.steps))
     if rank == 0:
         best = min(v["frac"] for k, v in res.items() if isinstance(v, dict))
-        line = {"metric": "PBSA score/update achieved HBM bandwidth at bandwidth scale",
+        line = {"metric": "PBSA HBM-bound calls: achieved HBM bandwidth at bandwidth scale "
+                          "(lowest of the calls)",
                 "value": round(best, 4), "unit": "fraction of measured HBM copy GB/s",
                 "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
                 "dtype": "bf16", "data": "synthetic (seeded N(0,1))",
                 "config": {"workload": "score_blocks on the trainable shape; update_memory "
-                                       "filling 128 slots of B2 H12", "parallelism": "replicas"},
+                                       "filling 128 slots of B2 H12; append_chunk of a "
+                                       "32 760-token chunk, B2 H12", "parallelism": "replicas"},
                 "calls": res, "peak_kind": pk_kind}
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -42,6 +42,8 @@ class PbsaRouteArgs(ctypes.Structure):
 SIGNATURES = {
     "pbsa_score_blocks": (c_int, [P, c_void_p, c_int, c_void_p, c_int, c_void_p, c_void_p, c_int,
                                   c_void_p, c_void_p, c_void_p, c_void_p, c_void_p]),
+    "pbsa_append_chunk": (c_int, [P, c_void_p, c_void_p, c_int, c_int, c_void_p, c_void_p, c_int,
+                                  c_void_p, c_void_p, c_void_p, c_void_p, c_void_p]),
     "pbsa_update_memory_workspace": (c_size_t, [P, c_int, c_int]),
     "pbsa_update_memory": (c_int, [P, c_void_p, c_void_p, c_int, c_void_p, c_void_p, c_void_p,
                                    c_int, c_int, c_void_p, c_void_p, c_void_p, c_void_p, c_int,

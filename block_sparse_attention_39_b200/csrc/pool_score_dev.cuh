@@ -70,6 +70,45 @@ struct Vec16<float> {
   }
 };
 
+// Column sums of rows [0, n) of a block staged in shared memory (rows of D
+// elements of T, 16-byte chunks), reduced to one partial row per warp in
+// rb[8][D].  Every thread of the 256-thread CTA calls it; the caller
+// synchronises before row_mean() reads rb.  Shared by the pooling of
+// pbsa_score_blocks and pbsa_append_chunk, so both give the same means.
+template <typename T, int D>
+__device__ __forceinline__ void row_sums(const uint8_t* stage, int n, float* rb) {
+  constexpr int EPC = Vec16<T>::EPC;
+  constexpr int CPR = D / EPC;
+  constexpr int RPP = kPoolThreads / CPR;
+  constexpr int ROW = D * static_cast<int>(sizeof(T));
+  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  const int c = t % CPR, rg = t / CPR;
+  float acc[EPC];
+#pragma unroll
+  for (int e = 0; e < EPC; ++e) acc[e] = 0.f;
+#pragma unroll 4
+  for (int r = rg; r < n; r += RPP) Vec16<T>::add(stage + r * ROW + c * 16, acc);
+#pragma unroll
+  for (int off = CPR; off < 32; off <<= 1) {
+#pragma unroll
+    for (int e = 0; e < EPC; ++e) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], off);
+  }
+  if (lane < CPR) {
+#pragma unroll
+    for (int e = 0; e < EPC; ++e) rb[warp * D + lane * EPC + e] = acc[e];
+  }
+}
+
+// Mean of column t (t < D) from the per-warp partial rows.
+template <int D>
+__device__ __forceinline__ float row_mean(const float* rb, int n) {
+  const int t = threadIdx.x;
+  float sum = 0.f;
+#pragma unroll
+  for (int w = 0; w < kPoolThreads / 32; ++w) sum += rb[w * D + t];
+  return n > 0 ? sum / static_cast<float>(n) : 0.f;
+}
+
 // Where item `it` (flattened over (b,h) x [query blocks, listed key blocks])
 // reads its rows and where its mean goes: `out` >= 0 is an offset into q_bar,
 // `out` <= -2 is the offset -(out + 2) into k_bar, -1 means no output (an
@@ -107,7 +146,6 @@ template <typename T, int D>
 __device__ void pool_phase(const PoolArgs& a, int cta, int G, uint8_t* smem) {
   constexpr int EPC = Vec16<T>::EPC;
   constexpr int CPR = D / EPC;                 // 16-byte chunks per row
-  constexpr int RPP = kPoolThreads / CPR;      // rows per pass
   constexpr int ROW = D * static_cast<int>(sizeof(T));
   static_assert(CPR <= 32 && (32 % CPR) == 0, "chunks per row must divide a warp");
   const int S = a.stages;
@@ -175,7 +213,6 @@ __device__ void pool_phase(const PoolArgs& a, int cta, int G, uint8_t* smem) {
     for (int k = 0; k < first; ++k) issue(k);
     issued = first;
   }
-  const int c = t % CPR, rg = t / CPR;
   bool ok = true;
   for (int k = 0; k < mine; ++k) {
     const int s = k % S;
@@ -184,33 +221,16 @@ __device__ void pool_phase(const PoolArgs& a, int cta, int G, uint8_t* smem) {
     if (__syncthreads_or(!ok)) { ok = false; break; }
     const int n = s_n[s];
     const long oo = s_out[s];
-    float acc[EPC];
-#pragma unroll
-    for (int e = 0; e < EPC; ++e) acc[e] = 0.f;
-    const uint8_t* stage = smem + s * stage_bytes;
-#pragma unroll 4
-    for (int r = rg; r < n; r += RPP) Vec16<T>::add(stage + r * ROW + c * 16, acc);
-#pragma unroll
-    for (int off = CPR; off < 32; off <<= 1) {
-#pragma unroll
-      for (int e = 0; e < EPC; ++e) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], off);
-    }
     float* rb = red + (k & 1) * 8 * D;
-    if (lane < CPR) {
-#pragma unroll
-      for (int e = 0; e < EPC; ++e) rb[warp * D + lane * EPC + e] = acc[e];
-    }
+    row_sums<T, D>(smem + s * stage_bytes, n, rb);
     __syncthreads();   // stage s fully read; partial sums of item k complete
     if (t == 0 && k + S < mine) {
       issue(k + S);
       ++issued;
     }
     if (t < D && oo != -1) {
-      float sum = 0.f;
-#pragma unroll
-      for (int w = 0; w < kPoolThreads / 32; ++w) sum += rb[w * D + t];
       float* out = oo >= 0 ? a.q_bar + oo : a.k_bar + (-(oo + 2));
-      out[t] = n > 0 ? sum / static_cast<float>(n) : 0.f;
+      out[t] = row_mean<D>(rb, n);
     }
   }
   // on a time-out, wait for the copies still in flight before the CTA exits:

@@ -59,6 +59,7 @@ class PbsaLayer:
         self.rws = torch.zeros(K.route_workspace(self.d, P, self.max_cand), dtype=torch.uint8,
                                device=dev)
         self._ids = {}
+        self._no_ids = torch.zeros(0, dtype=torch.int32, device=dev)
         if self.tdtype != torch.bfloat16:
             # attention runs on bf16 copies of an fp32 cache (R17)
             self.q16 = torch.zeros(B, H, w.chunk_tokens, D, dtype=torch.bfloat16, device=dev)
@@ -113,6 +114,15 @@ class PbsaLayer:
                 self.vpool[:, :, pid, lens[j]:] = 0
         self.set_chunk_meta(t)
 
+    def append(self, t, k_chunk, v_chunk, stream=None):
+        """Chunk t's K/V [B,H,T_c,D] into its blocks with their pooled keys in the
+        same pass (pbsa_append_chunk); the next score call then pools only the
+        queries (``step(t, appended=True)``)."""
+        w = self.w
+        K.append_chunk(self.d, k_chunk, v_chunk, w.chunk_tokens, t * w.chunk_tokens, self.kpool,
+                       self.vpool, self.NB, self.chunk_ids(t), self.blk_len, self.blk_pos,
+                       self.k_bar, stream)
+
     # ------------------------------------------------------------ the hot path
     def score(self, t, pool_ids=None, stream=None):
         w = self.w
@@ -161,8 +171,9 @@ class PbsaLayer:
         cs = self.ids(key + ("src",), [g for c in chunks for g in w.chunk_global_ids(c)])
         return ci, cs
 
-    def route(self, t, stream=None):
-        """Score -> update -> select for chunk t in one call (pbsa_route_step)."""
+    def route(self, t, stream=None, appended=False):
+        """Score -> update -> select for chunk t in one call (pbsa_route_step).
+        appended: the chunk's pooled keys were written by append()."""
         w = self.w
         pids = self.chunk_ids(t)
         ci, cs = self.candidates(t)
@@ -171,7 +182,7 @@ class PbsaLayer:
         K.route_step(self.d, self.rws, stream,
                      q=self.q, Tq=w.chunk_tokens, kpool=self.kpool, vpool=self.vpool, NB=self.NB,
                      blk_len=self.blk_len, blk_pos=self.blk_pos, pool_ids=pids,
-                     n_pool=pids.numel(), q_bar=self.q_bar, k_bar=self.k_bar, scores=self.scores,
+                     n_pool=0 if appended else pids.numel(), q_bar=self.q_bar, k_bar=self.k_bar, scores=self.scores,
                      mem_score=self.mem, P=self.P, n_sink=w.n_sink,
                      slot_src=self.slot_src if self.P else None,
                      slot_w=self.slot_w if self.P else None,
@@ -180,15 +191,17 @@ class PbsaLayer:
                      mem_ids=self.mem_ids, n_mem=self.P, mask=w.mask, q_pos0=t * w.chunk_tokens,
                      idx=self.idx, cnt=self.cnt, Amax=self.Amax)
 
-    def step(self, t, stream=None, fused=False):
+    def step(self, t, stream=None, fused=False, appended=False):
         """Score -> update -> select -> attend for chunk t (its Q already in self.q,
         its K/V already in the pool).  fused: the first three as one routing call
         (pbsa_route_step); the default is the per-call path, which is the faster
-        schedule on the decode and rollout shapes."""
+        schedule on the decode and rollout shapes.  appended: the chunk's K/V
+        came in through append(), so its pooled keys exist and only the queries
+        are pooled."""
         if fused:
-            self.route(t, stream=stream)
+            self.route(t, stream=stream, appended=appended)
         else:
-            self.score(t, stream=stream)
+            self.score(t, pool_ids=self._no_ids if appended else None, stream=stream)
             ci, cs = self.candidates(t)
             self.update(ci, cs, stream=stream)
             self.select(t, stream=stream)

@@ -65,6 +65,13 @@ def score_blocks(d: PbsaDims, q, Tq, kpool, NB, blk_len, pool_ids, n_pool, q_bar
         _p(k_bar), _p(scores), _p(mem_score), _s(stream)))
 
 
+def append_chunk(d: PbsaDims, k, v, Tc, pos0, kpool, vpool, NB, blk_ids, blk_len, blk_pos, k_bar,
+                 stream=None):
+    _check("pbsa_append_chunk", lib().pbsa_append_chunk(
+        ctypes.byref(d), _p(k), _p(v), Tc, pos0, _p(kpool), _p(vpool), NB, _p(blk_ids),
+        _p(blk_len), _p(blk_pos), _p(k_bar), _s(stream)))
+
+
 def update_memory_workspace(d: PbsaDims, P: int, n_cand: int) -> int:
     return int(lib().pbsa_update_memory_workspace(ctypes.byref(d), P, n_cand))
 

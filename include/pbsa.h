@@ -109,6 +109,32 @@ int pbsa_score_blocks(const pbsa_dims* dims, const void* q, int Tq,
                       void* stream);
 
 /* ---------------------------------------------------------------------------
+ * a0: KV append with block compression fused in.
+ * Passage: gist.science/es section 2, PBSA item "Compresión de Bloques" (the
+ * pooled representative of each block) and item "Optimización" (selective KV
+ * cache updates are part of the kernel's job).
+ *
+ * The chunk's rows t = 0..Tc-1 fall into blocks c = t / bs (nb = ceil(Tc/bs)
+ * of them; the last may be partial).  Chunk block c goes to pool block
+ * blk_ids[c], for every (b,h):
+ *   kpool[b,h,blk_ids[c], r] = k[b,h,c*bs + r]   for r < n_c = min(bs, Tc - c*bs)
+ *   vpool[b,h,blk_ids[c], r] = v[b,h,c*bs + r]   (rows r >= n_c are zeroed)
+ *   blk_len[b,h,blk_ids[c]] = n_c,  blk_pos[b,h,blk_ids[c]] = pos0 + c*bs
+ *   k_bar[b,h,blk_ids[c]]   = mean of the n_c rows written (fp32), the same
+ *                             value pbsa_score_blocks gives for that block
+ * so a following pbsa_score_blocks needs no pool_ids for the chunk's blocks.
+ *
+ * k, v: dtype of dims, [B,H,Tc,D] contiguous.  kpool, vpool: [B,H,NB,bs,D].
+ * blk_len, blk_pos: int32 [B,H,NB].  k_bar: fp32 [B,H,NB,D].  blk_ids: device
+ * int32 [nb], distinct, each in [0, NB) (an id outside that range sets the
+ * device status to PBSA_ERR_ARG and its block is skipped).  k, v, kpool, vpool
+ * 16-byte aligned.  Nothing is allocated; the call is asynchronous on stream.
+ * ------------------------------------------------------------------------- */
+int pbsa_append_chunk(const pbsa_dims* dims, const void* k, const void* v, int Tc, int pos0,
+                      void* kpool, void* vpool, int NB, const int32_t* blk_ids,
+                      int32_t* blk_len, int32_t* blk_pos, float* k_bar, void* stream);
+
+/* ---------------------------------------------------------------------------
  * a3: persistent-memory update (Top-C retention, sinks, evict or mean-merge).
  * Passage: gist.science/es section 2 "Arquitectura Propuesta", items "Memoria
  * Persistente", "Bloques Sumidero", "Bloques Dinámicos", "Mecanismo de

@@ -144,3 +144,21 @@ def test_route_rejects_bad_arguments_without_launch():
     assert lib.pbsa_route_workspace(ctypes.byref(d), 0, 0) == 256
     assert (lib.pbsa_route_workspace(ctypes.byref(d), 24, 111)
             == 256 + lib.pbsa_update_memory_workspace(ctypes.byref(d), 24, 111))
+
+
+def test_append_rejects_bad_arguments_without_launch():
+    lib = _lib.lib()
+    d = _d()
+    fake = ctypes.c_void_p(256)       # never dereferenced: validation fails first
+    # NULL buffers
+    assert lib.pbsa_append_chunk(ctypes.byref(d), NULL, NULL, 300, 0, NULL, NULL, 8, NULL, NULL,
+                                 NULL, NULL, NULL) == -1
+    # the chunk (3 blocks of 128) does not fit a 2-block pool
+    assert lib.pbsa_append_chunk(ctypes.byref(d), fake, fake, 300, 0, fake, fake, 2, fake, fake,
+                                 fake, fake, NULL) == -2
+    # empty chunk
+    assert lib.pbsa_append_chunk(ctypes.byref(d), fake, fake, 0, 0, fake, fake, 8, fake, fake,
+                                 fake, fake, NULL) == -2
+    # misaligned K rows
+    assert lib.pbsa_append_chunk(ctypes.byref(d), ctypes.c_void_p(264), fake, 300, 0, fake, fake,
+                                 8, fake, fake, fake, fake, NULL) == -3
