@@ -1,6 +1,6 @@
 // a1 + a2: block pooling and coarse block scoring, as two kernels per call:
-// a persistent pooling grid (two CTAs per SM) and one scoring CTA per
-// (b,h, 16 key blocks).  The device code is in pool_score_dev.cuh.
+// a persistent pooling grid (two CTAs per SM) and one 64-thread scoring CTA
+// per (b,h, 32 query blocks, 32 key blocks) tile of S.  The device code is in pool_score_dev.cuh.
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 
@@ -22,11 +22,13 @@ __global__ void __launch_bounds__(kPoolThreads) pool_kernel(PoolArgs a) {
 }
 
 template <int D>
-__global__ void __launch_bounds__(256) score_kernel(ScoreArgs a) {
+__global__ void __launch_bounds__(kScoreThreads) score_kernel(ScoreArgs a) {
   extern __shared__ __align__(16) float ssm[];
   pdl_wait();
   pdl_trigger();
-  score_item<D>(a, blockIdx.y, static_cast<int>(blockIdx.x), ssm);
+  const int n_jblk = (a.NB + kScoreTile - 1) / kScoreTile;
+  const int x = static_cast<int>(blockIdx.x);
+  score_item<D, kScoreTile>(a, blockIdx.y, x % n_jblk, x / n_jblk, ssm);
 }
 
 template <typename T, int D>
@@ -52,17 +54,17 @@ int launch_pool(PoolArgs a, cudaStream_t s) {
 
 template <int D>
 int launch_score(const ScoreArgs& a, int BH, cudaStream_t s) {
-  const size_t smem = score_smem_bytes<D>(a.nQB);
+  const size_t smem = score_smem_bytes<D, kScoreTile>();
   static bool attr_set[64] = {false};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !attr_set[dev]) {
     cudaFuncSetAttribute(score_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         static_cast<int>(kScoreQI * D * 4 + kScoreTileMax * kScoreJ * 4));
+                         static_cast<int>(smem));
     attr_set[dev] = true;
   }
-  dim3 grid((a.NB + kScoreJ - 1) / kScoreJ, BH);
-  cudaError_t e = launch(score_kernel<D>, grid, dim3(256), smem, s, a);
+  dim3 grid(((a.NB + kScoreTile - 1) / kScoreTile) * ((a.nQB + kScoreTile - 1) / kScoreTile), BH);
+  cudaError_t e = launch(score_kernel<D>, grid, dim3(kScoreThreads), smem, s, a);
   if (e != cudaSuccess) {
     set_error(std::string("score_kernel: ") + cudaGetErrorString(e));
     return PBSA_ERR_CUDA;

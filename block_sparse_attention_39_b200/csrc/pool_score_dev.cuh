@@ -260,9 +260,13 @@ __host__ __device__ inline int pool_stages(int bs) {
   return st < 2 ? 2 : (st > 4 ? 4 : st);
 }
 
-constexpr int kScoreJ = 16;     // key blocks per CTA
-constexpr int kScoreQI = 64;    // query blocks staged per pass
-constexpr int kScoreTileMax = 1024;   // query blocks whose S columns stay in shared memory
+// Tiles of S: the per-call scoring kernel runs 32 x 32 tiles on 64-thread
+// CTAs (enough CTAs to cover the SMs on a decode step's few hundred tiles);
+// the fused routing kernel runs 64 x 64 tiles on its 256 threads.  Every
+// score and memory score is computed in the same order in both, so the two
+// give the same bits.
+constexpr int kScoreTile = 32, kScoreThreads = 64;
+constexpr int kRouteScoreTile = 64;
 
 struct ScoreArgs {
   const float* q_bar;
@@ -273,88 +277,156 @@ struct ScoreArgs {
   float scale;
 };
 
-// Scores of key blocks [16 jblk, 16 jblk + 16) against every query block of
-// head bh, and their memory scores.  `ssm` holds score_smem_bytes() bytes.
+// Row pitch (floats) of the staged q_bar / k_bar tiles: D + 4 puts the 8
+// rows a quarter-warp reads at once on distinct bank groups.
 template <int D>
-__device__ void score_item(const ScoreArgs& a, long bh, int jblk, float* ssm) {
-  const int QI = min(a.nQB, kScoreQI);
-  float4* qs = reinterpret_cast<float4*>(ssm);            // [QI][D/4]
-  float* st = ssm + QI * D;                               // [nQB][16] when kept
-  const bool keep = a.nQB <= kScoreTileMax;
-  const int j0 = jblk * kScoreJ;
-  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
-  const int jj = lane & 15, half = lane >> 4;
-  const int j = j0 + jj;
-  // half `half` of pooled key j: float4 number 2m + half, m < D/8
-  constexpr int NV = D / 8;
-  float4 kr[NV];
-  {
-    const float4* krow =
-        reinterpret_cast<const float4*>(a.k_bar + (bh * a.NB + min(j, a.NB - 1)) * D);
+__host__ __device__ constexpr int score_pitch() { return D + 4; }
+
+// Stage rows [0, n) of a [*, D] fp32 matrix as the TR rows of a padded tile
+// (NT threads): 16-byte asynchronous copies (cp.async, no registers held, all
+// of a thread's copies in flight at once), zeros for rows past n.  The caller
+// waits with score_stage_wait() and then synchronises the CTA.
+template <int D, int TR, int NT>
+__device__ __forceinline__ void score_stage(float* tile, const float* src, int n) {
+  constexpr int PER = TR * (D / 4) / NT;
+  static_assert(PER * NT == TR * (D / 4), "tile must split evenly over the threads");
+  const int t = threadIdx.x;
 #pragma unroll
-    for (int m = 0; m < NV; ++m) kr[m] = krow[2 * m + half];
-  }
-  const float4* qsrc = reinterpret_cast<const float4*>(a.q_bar + bh * a.nQB * D);
-  for (int i0 = 0; i0 < a.nQB; i0 += QI) {
-    const int ni = min(QI, a.nQB - i0);
-    __syncthreads();
-    // all of a thread's loads in flight together (8 per batch)
-    for (int e0 = 0; e0 < ni * (D / 4); e0 += 256 * 8) {
-      float4 v[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int e = e0 + u * 256 + t;
-        if (e < ni * (D / 4)) v[u] = qsrc[i0 * (D / 4) + e];
-      }
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int e = e0 + u * 256 + t;
-        if (e < ni * (D / 4)) qs[e] = v[u];
-      }
-    }
-    __syncthreads();
-    for (int ii = warp; ii < ni; ii += 8) {
-      const float4* qr = qs + ii * (D / 4);
-      float s0 = 0.f, s1 = 0.f;
-#pragma unroll
-      for (int m = 0; m < NV; ++m) {
-        const float4 q = qr[2 * m + half];
-        s0 = fmaf(q.x, kr[m].x, s0);
-        s1 = fmaf(q.y, kr[m].y, s1);
-        s0 = fmaf(q.z, kr[m].z, s0);
-        s1 = fmaf(q.w, kr[m].w, s1);
-      }
-      float s = s0 + s1;
-      s += __shfl_xor_sync(0xffffffffu, s, 16);
-      s *= a.scale;
-      if (half == 0 && j < a.NB) {
-        a.scores[(bh * a.nQB + i0 + ii) * a.NB + j] = s;
-        if (keep) st[(i0 + ii) * kScoreJ + jj] = s;
-      }
-    }
-  }
-  __syncthreads();
-  // memory score of every query chunk: mean of S over its query blocks, in
-  // block order
-  for (int e = t; e < a.groups * kScoreJ; e += 256) {
-    const int g = e / kScoreJ, c = e % kScoreJ, jc = j0 + c;
-    if (jc >= a.NB) continue;
-    const int i_lo = g * a.per_group, i_hi = min(a.nQB, (g + 1) * a.per_group);
-    float m = 0.f;
-    if (keep) {
-      for (int i = i_lo; i < i_hi; ++i) m += st[i * kScoreJ + c];
+  for (int u = 0; u < PER; ++u) {
+    const int e = t + u * NT, row = e / (D / 4), c4 = e % (D / 4);
+    float* dst = tile + row * score_pitch<D>() + c4 * 4;
+    if (row < n) {
+      asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(smem_u32(dst)),
+                   "l"(src + static_cast<long>(e) * 4)
+                   : "memory");
     } else {
-      for (int i = i_lo; i < i_hi; ++i) m += a.scores[(bh * a.nQB + i) * a.NB + jc];
+      *reinterpret_cast<float4*>(dst) = make_float4(0.f, 0.f, 0.f, 0.f);
     }
-    a.mem[(bh * a.groups + g) * a.NB + jc] = m / static_cast<float>(i_hi - i_lo);
+  }
+}
+__device__ __forceinline__ void score_stage_wait() {
+  asm volatile("cp.async.commit_group;\n" ::: "memory");
+  asm volatile("cp.async.wait_group 0;\n" ::: "memory");
+}
+
+// One T x T tile of S: query blocks [T itile, +T) against key blocks
+// [T jblk, +T) of head bh, plus the memory scores of the query chunks that
+// start inside the tile's rows.  Called by all NT = T*T/16 threads of the CTA.
+//
+// The tile is a small fp32 GEMM on the CUDA cores (K = D is short, and the
+// scores are compared against a selection threshold, so no reduced-precision
+// tensor-core inputs): thread (ty, tx) of the (T/4) x (T/4) grid owns rows
+// ty + (T/4) k and columns tx + (T/4) l (k, l < 4); every score is one fmaf
+// chain over d = 0 .. D-1 in order, times scale.
+//
+// The memory score of chunk g is the mean of its scores over its query blocks.
+// The scores are linear in the pooled query, so that mean is computed as
+// scale * <mean of the chunk's pooled queries, k_bar_j> (equal up to rounding):
+// the chunk's mean query (sum in block order, fp32, then one divide), then one
+// dot per key block, split over four lanes (float4 number p + 4m to lane p)
+// and combined as (s0 + s1) + (s2 + s3).  The tile holding the chunk's first
+// query block does it, so no tile waits on another.
+template <int D, int T>
+__device__ void score_item(const ScoreArgs& a, long bh, int jblk, int itile, float* ssm) {
+  constexpr int PT = score_pitch<D>();
+  constexpr int G4 = T / 4, NT = G4 * G4;
+  float* ks = ssm;                                         // [T][PT]
+  float* qs = ks + T * PT;                                 // [T][PT]
+  float* qm = qs + T * PT;                                 // [D] a chunk's mean query
+  const int t = threadIdx.x, tx = t % G4, ty = t / G4;
+  const int j0 = jblk * T, i0 = itile * T;
+  const int nj = min(T, a.NB - j0), ni = min(T, a.nQB - i0);
+  const float* qrows = a.q_bar + bh * a.nQB * D;
+  __syncthreads();                    // the previous item's readers are done
+  score_stage<D, T, NT>(ks, a.k_bar + (bh * a.NB + j0) * D, nj);
+  score_stage<D, T, NT>(qs, qrows + static_cast<long>(i0) * D, ni);
+  score_stage_wait();
+  __syncthreads();
+  float acc[4][4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k)
+#pragma unroll
+    for (int l = 0; l < 4; ++l) acc[k][l] = 0.f;
+#pragma unroll 4
+  for (int d = 0; d < D; d += 4) {
+    float4 q[4], kk[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) q[k] = *reinterpret_cast<const float4*>(qs + (ty + G4 * k) * PT + d);
+#pragma unroll
+    for (int l = 0; l < 4; ++l) kk[l] = *reinterpret_cast<const float4*>(ks + (tx + G4 * l) * PT + d);
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+#pragma unroll
+      for (int l = 0; l < 4; ++l) {
+        float s = acc[k][l];
+        s = fmaf(q[k].x, kk[l].x, s);
+        s = fmaf(q[k].y, kk[l].y, s);
+        s = fmaf(q[k].z, kk[l].z, s);
+        s = fmaf(q[k].w, kk[l].w, s);
+        acc[k][l] = s;
+      }
+  }
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int r = ty + G4 * k;
+#pragma unroll
+    for (int l = 0; l < 4; ++l) {
+      const int c = tx + G4 * l;
+      if (r < ni && c < nj) a.scores[(bh * a.nQB + i0 + r) * a.NB + j0 + c] = acc[k][l] * a.scale;
+    }
+  }
+  // chunks whose first query block is in rows [i0, i0 + ni)
+  const int g_lo = (i0 + a.per_group - 1) / a.per_group;
+  const int g_hi = min(a.groups, (i0 + ni + a.per_group - 1) / a.per_group);
+  for (int g = g_lo; g < g_hi; ++g) {
+    const int r_lo = g * a.per_group, r_hi = min(a.nQB, r_lo + a.per_group);
+    const int r_mid = min(r_hi, i0 + ni);          // rows below r_mid are staged
+    {
+      // the DPT columns of a thread summed side by side, so the rows past the
+      // staged tile cost one round of loads, not DPT
+      constexpr int DPT = (D + NT - 1) / NT;
+      float sum[DPT];
+#pragma unroll
+      for (int u = 0; u < DPT; ++u) sum[u] = 0.f;
+      for (int i = r_lo; i < r_mid; ++i) {
+#pragma unroll
+        for (int u = 0; u < DPT; ++u)
+          if (t + u * NT < D) sum[u] += qs[(i - i0) * PT + t + u * NT];
+      }
+#pragma unroll 8
+      for (int i = r_mid; i < r_hi; ++i) {
+#pragma unroll
+        for (int u = 0; u < DPT; ++u)
+          if (t + u * NT < D) sum[u] += qrows[static_cast<long>(i) * D + t + u * NT];
+      }
+#pragma unroll
+      for (int u = 0; u < DPT; ++u)
+        if (t + u * NT < D) qm[t + u * NT] = sum[u] / static_cast<float>(r_hi - r_lo);
+    }
+    __syncthreads();
+    const int p = t & 3;
+    for (int c = t >> 2; c < T; c += NT / 4) {
+      float s = 0.f;
+#pragma unroll
+      for (int m = 0; m < D / 16; ++m) {
+        const float4 x = *reinterpret_cast<const float4*>(qm + (p + 4 * m) * 4);
+        const float4 y = *reinterpret_cast<const float4*>(ks + c * PT + (p + 4 * m) * 4);
+        s = fmaf(x.x, y.x, s);
+        s = fmaf(x.y, y.y, s);
+        s = fmaf(x.z, y.z, s);
+        s = fmaf(x.w, y.w, s);
+      }
+      s += __shfl_xor_sync(0xffffffffu, s, 1);
+      s += __shfl_xor_sync(0xffffffffu, s, 2);
+      if (p == 0 && c < nj) a.mem[(bh * a.groups + g) * a.NB + j0 + c] = s * a.scale;
+    }
+    __syncthreads();                  // qm free for the next chunk
   }
 }
 
-template <int D>
-__host__ __device__ inline size_t score_smem_bytes(int nQB) {
-  const int QI = nQB < kScoreQI ? nQB : kScoreQI;
-  return static_cast<size_t>(QI) * D * sizeof(float) +
-         (nQB <= kScoreTileMax ? static_cast<size_t>(nQB) * kScoreJ * 4 : 0);
+template <int D, int T>
+__host__ __device__ inline size_t score_smem_bytes() {
+  return static_cast<size_t>(2 * T * score_pitch<D>() + D) * sizeof(float);
 }
 
 }  // namespace dev

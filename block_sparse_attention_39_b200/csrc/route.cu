@@ -45,7 +45,7 @@ struct RouteParams {
   int32_t* slot_src;
   float* slot_w;
   unsigned long long* bar;   // [0] arrivals, [1] exits
-  int do_update, n_score_items, n_jblk, BH, P, n_rows, nQB;
+  int do_update, n_score_items, n_jblk, n_itile, BH, P, n_rows, nQB;
   int* status;
   int64_t limit_ns;
 };
@@ -73,6 +73,9 @@ __device__ __forceinline__ void grid_sync(const RouteParams& r, unsigned long lo
   __syncthreads();
 }
 
+static_assert(kRouteScoreTile * kRouteScoreTile / 16 == kRouteThreads,
+              "one 4 x 4 block of the score tile per routing thread");
+
 template <typename T, int D, int W, int U>
 __global__ void __launch_bounds__(kRouteThreads, 2) route_kernel(RouteParams r) {
   extern __shared__ __align__(128) uint8_t smem[];
@@ -83,9 +86,12 @@ __global__ void __launch_bounds__(kRouteThreads, 2) route_kernel(RouteParams r) 
   pool_phase<T, D>(r.pool, cta, G, smem);
   grid_sync(r, target += G);
 
-  // a2: scores and memory scores, one (b,h, 16 key blocks) item at a time
-  for (int it = cta; it < r.n_score_items; it += G)
-    score_item<D>(r.score, it / r.n_jblk, it % r.n_jblk, reinterpret_cast<float*>(smem));
+  // a2: scores and memory scores, one (b,h, 64 x 64 tile of S) item at a time
+  for (int it = cta; it < r.n_score_items; it += G) {
+    const int per_bh = r.n_jblk * r.n_itile, x = it % per_bh;
+    score_item<D, kRouteScoreTile>(r.score, it / per_bh, x % r.n_jblk, x / r.n_jblk,
+                                   reinterpret_cast<float*>(smem));
+  }
   grid_sync(r, target += G);
 
   // a3: plan per (b,h), then stash (merge) and apply per (slot, b,h)
@@ -137,7 +143,7 @@ __global__ void __launch_bounds__(kRouteThreads, 2) route_kernel(RouteParams r) 
 template <typename T, int D>
 size_t route_smem(const RouteParams& r) {
   size_t m = pool_smem_bytes<T, D>(r.pool.stages, r.pool.bs);
-  m = std::max(m, score_smem_bytes<D>(r.nQB));
+  m = std::max(m, score_smem_bytes<D, kRouteScoreTile>());
   if (r.do_update) {
     size_t plan = (sizeof(PlanSmem) + 15) / 16 * 16;
     if (r.upd.policy == PBSA_MERGE_MEAN) plan += merge_key_smem(r.P, D);
@@ -317,8 +323,9 @@ extern "C" int pbsa_route_step(const pbsa_dims* d, const pbsa_route_args* a, voi
   r.slot_src = a->slot_src; r.slot_w = a->slot_w;
   r.bar = reinterpret_cast<unsigned long long*>(ws);
   r.do_update = do_update ? 1 : 0;
-  r.n_jblk = (a->NB + kScoreJ - 1) / kScoreJ;
-  r.n_score_items = BH * r.n_jblk;
+  r.n_jblk = (a->NB + kRouteScoreTile - 1) / kRouteScoreTile;
+  r.n_itile = (nQB + kRouteScoreTile - 1) / kRouteScoreTile;
+  r.n_score_items = BH * r.n_jblk * r.n_itile;
   r.BH = BH; r.P = a->P; r.n_rows = BH * nQB; r.nQB = nQB;
   r.status = status; r.limit_ns = wait_limit_ns();
 

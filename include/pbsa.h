@@ -97,7 +97,9 @@ typedef struct {
  *                      a block of length 0 pools to zero)
  *   scores[b,h,i,j]  = scale * <q_bar[b,h,i], k_bar[b,h,j]>  for all j < NB
  *   mem_score[b,h,g,j] = mean of scores[b,h,i,j] over the query blocks i of
- *                      query chunk g (one chunk, g = 0, when dims.q_chunk = 0)
+ *                      query chunk g (one chunk, g = 0, when dims.q_chunk = 0),
+ *                      computed as scale * <mean of those q_bar[b,h,i],
+ *                      k_bar[b,h,j]>, which equals it up to rounding
  *
  * q, kpool: dtype of dims (bf16 or fp32).  pool_ids: device int32 [n_pool],
  * the same list for every (b,h); n_pool may be 0.  Outputs are overwritten.
