@@ -284,6 +284,10 @@ extern "C" int pbsa_route_step(const pbsa_dims* d, const pbsa_route_args* a, voi
   }
   const long n_items = static_cast<long>(d->B) * d->H * (nQB + a->n_pool);
   PBSA_CHECK_ARG(n_items < (1L << 31), PBSA_ERR_SHAPE, "route_step: too many blocks to pool");
+  const long n_score_items = static_cast<long>(d->B) * d->H *
+                             ((a->NB + kRouteScoreTile - 1) / kRouteScoreTile) *
+                             ((nQB + kRouteScoreTile - 1) / kRouteScoreTile);
+  PBSA_CHECK_ARG(n_score_items < (1L << 31), PBSA_ERR_SHAPE, "route_step: too many score tiles");
   int* status = device_status_ptr();
   PBSA_CHECK_ARG(status != nullptr, PBSA_ERR_CUDA, "route_step: no device status word");
 
