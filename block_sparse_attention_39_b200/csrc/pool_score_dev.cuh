@@ -13,11 +13,10 @@
 // blocks in flight; the rows are summed in fp32 from shared memory with
 // 128-bit reads and a warp-shuffle + shared-memory reduction.  Every input
 // byte is read once.
-// score_item: one (b,h, 16 key blocks) item.  Each thread keeps half of one
-// pooled key in registers; the query-block means are staged in shared memory;
-// S is written row by row and the memory score of every query chunk (the mean
-// of S over the chunk's query blocks, summed in block order) is formed from a
-// shared-memory copy of the item's S columns.
+// score_item: one square tile of S (b,h, T query blocks x T key blocks) as a
+// small fp32 GEMM on the CUDA cores, from q_bar / k_bar rows staged by cp.async;
+// the memory scores of the query chunks that start in the tile come from the
+// chunk's mean pooled query, so tiles are independent of one another.
 #pragma once
 
 #include <cuda_runtime.h>
