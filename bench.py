@@ -223,7 +223,7 @@ class DecodeRunner:
         L = self.L
         if fused is None:
             fused = self.fused
-        pids = L._no_ids if appended else None
+        pids = L.no_ids if appended else None
         calls = ([lambda: L.route(self.t, appended=appended)] if fused else
                  [lambda: L.score(self.t, pool_ids=pids), lambda: L.update(*self.cand),
                   lambda: L.select(self.t)])
@@ -687,7 +687,7 @@ def bench_append(torch, runner, pk, reps=20):
     out["append_chunk, decode chunk"] = entry(append_traffic(w.B * w.H, w.chunk_tokens, w.nb_c, w.bs,
                                                       w.D), ms)
     out["score_blocks, keys pooled by the append (queries only)"] = {
-        "ms": round(_graph_timed(torch, lambda: L.score(t, pool_ids=L._no_ids), reps,
+        "ms": round(_graph_timed(torch, lambda: L.score(t, pool_ids=L.no_ids), reps,
                                  pre=flush.zero_), 5)}
     out["score_blocks, pooling the chunk's keys itself"] = {
         "ms": round(_graph_timed(torch, lambda: L.score(t), reps, pre=flush.zero_), 5)}

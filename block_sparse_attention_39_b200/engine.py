@@ -59,7 +59,8 @@ class PbsaLayer:
         self.rws = torch.zeros(K.route_workspace(self.d, P, self.max_cand), dtype=torch.uint8,
                                device=dev)
         self._ids = {}
-        self._no_ids = torch.zeros(0, dtype=torch.int32, device=dev)
+        # an empty id list: a score call that pools only the queries
+        self.no_ids = torch.zeros(0, dtype=torch.int32, device=dev)
         if self.tdtype != torch.bfloat16:
             # attention runs on bf16 copies of an fp32 cache (R17)
             self.q16 = torch.zeros(B, H, w.chunk_tokens, D, dtype=torch.bfloat16, device=dev)
@@ -201,7 +202,7 @@ class PbsaLayer:
         if fused:
             self.route(t, stream=stream, appended=appended)
         else:
-            self.score(t, pool_ids=self._no_ids if appended else None, stream=stream)
+            self.score(t, pool_ids=self.no_ids if appended else None, stream=stream)
             ci, cs = self.candidates(t)
             self.update(ci, cs, stream=stream)
             self.select(t, stream=stream)
