@@ -187,22 +187,21 @@ class DecodeRunner:
         self.torch = torch
         w = rank_workload(seed_offset)
         self.w = w
-        snap = PI.snapshot(w)
-        self.snap = snap
+        chunks = PI.snapshot_chunks(w)
+        self.chunks = chunks
         L = PbsaLayer(w)
+        self.lay = L.layout
         dev = torch.device("cuda")
 
         def st(x):
             return torch.from_numpy(np.ascontiguousarray(x)).to(dev).to(torch.bfloat16)
-        L.kpool.copy_(st(snap["kpool"]))
-        L.vpool.copy_(st(snap["vpool"]))
-        L.blk_len.copy_(torch.from_numpy(snap["blk_len"]).to(dev))
-        L.blk_pos.copy_(torch.from_numpy(snap["blk_pos"]).to(dev))
-        L.q.copy_(st(snap["q"]))
-        self.L = L
+        for t, (_, k, v) in chunks.items():
+            L.write_chunk(t, st(k), st(v))
         self.t = w.n_chunks - 1
+        L.q.copy_(st(chunks[self.t][0]))
+        self.L = L
         # pooled keys of every cached block (older blocks stay cached)
-        L.score(self.t, pool_ids=L.ids(("all",), snap["all_ids"]))
+        L.score(self.t, pool_ids=L.all_ids())
         L.reset_memory()
         self.cand = L.candidates(self.t)
         L.window_ids(self.t)
@@ -237,13 +236,10 @@ class DecodeRunner:
 
     def chunk_kv(self):
         """The step's chunk as the [B,H,T_c,D] K and V a caller appends."""
-        torch, w = self.torch, self.w
-        ids = w.chunk_phys_ids(self.t)
-
-        def rows(pool):
-            x = pool[:, :, ids].reshape(w.B, w.H, len(ids) * w.bs, w.D)[:, :, :w.chunk_tokens]
-            return torch.from_numpy(np.ascontiguousarray(x)).to(torch.bfloat16)
-        return rows(self.snap["kpool"]), rows(self.snap["vpool"])
+        torch = self.torch
+        _, k, v = self.chunks[self.t]
+        return (torch.from_numpy(np.ascontiguousarray(k)).to(torch.bfloat16),
+                torch.from_numpy(np.ascontiguousarray(v)).to(torch.bfloat16))
 
     def prologue(self):
         self.L.reset_memory()
@@ -254,7 +250,7 @@ class DecodeRunner:
         idx = L.idx.cpu().numpy()
         cnt = L.cnt.cpu().numpy()
         bl = L.blk_len.cpu().numpy()
-        lens = np.array(self.w.chunk_block_lens(), dtype=np.int64)
+        lens = np.array(self.lay.block_lens(), dtype=np.int64)
         total = 0
         for b in range(self.w.B):
             for h in range(self.w.H):
@@ -271,11 +267,11 @@ class DecodeRunner:
         BH = w.B * w.H
         el = 2
         rows_q = w.chunk_tokens
-        rows_k = sum(w.chunk_block_lens())                 # new chunk's valid key rows
-        NB = L.NB
+        rows_k = sum(self.lay.block_lens())                # new chunk's valid key rows
+        NB, nb_c = L.NB, self.lay.nb_c
         score = BH * (rows_q * w.D * el + rows_k * w.D * el          # Q and new K read
-                      + L.nQB * w.D * 4 + w.nb_c * w.D * 4         # q_bar, new k_bar written
-                      + (NB - w.nb_c) * w.D * 4                    # older k_bar read
+                      + L.nQB * w.D * 4 + nb_c * w.D * 4           # q_bar, new k_bar written
+                      + (NB - nb_c) * w.D * 4                      # older k_bar read
                       + L.nQB * NB * 4 + NB * 4)                   # S and m written
         src = L.slot_src.cpu().numpy()
         written = int((src >= 0).sum())                            # slots (re)written this step
@@ -327,7 +323,7 @@ class DecodeRunner:
         device time over the steps."""
         torch = self.torch
         L, w = self.L, self.w
-        hq = torch.from_numpy(self.snap["q"]).to(torch.bfloat16).pin_memory()
+        hq = torch.from_numpy(self.chunks[self.t][0]).to(torch.bfloat16).pin_memory()
         ck, cv = self.chunk_kv()
         hk, hv = ck.pin_memory(), cv.pin_memory()
         ho = [torch.empty(L.o.shape, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
@@ -461,7 +457,7 @@ def bench_train(torch, flush, reps=5):
     for t in (T.kpool, T.vpool):
         t.copy_(torch.randn(t.shape, generator=g, device="cuda").bfloat16())
     T.set_meta()
-    lens = np.array([n for c in range(w.n_chunks) for n in w.chunk_block_lens()], dtype=np.int64)
+    lens = np.array([n for c in range(w.n_chunks) for n in T.layout.block_lens()], dtype=np.int64)
     bl = T.blk_len.cpu().numpy()
     out = {"shape": f"B{w.B} H{w.H} D{w.D} bf16, {w.n_chunks} chunks x {w.chunk_tokens} tokens "
                     f"= {T.T} tokens, {T.NB} blocks of {w.bs}, chunk-causal"}
@@ -495,11 +491,11 @@ def bench_dense_comparators(torch, runner, flush, reps=10):
     """The decode inputs through the same attention kernel with full lists:
     the whole cache (185 blocks) and the sliding window alone (last 2 chunks)."""
     from block_sparse_attention_39_b200 import pbsa as K
-    L, w = runner.L, runner.w
+    L, w, lay = runner.L, runner.w, runner.lay
     out = {}
     for name, chunks in (("dense_full_cache", list(range(w.n_chunks))),
-                         ("dense_sliding_window", w.window_chunks(w.n_chunks - 1))):
-        ids = [p for c in chunks for p in w.chunk_phys_ids(c)]
+                         ("dense_sliding_window", lay.window_chunks(w.n_chunks - 1))):
+        ids = [p for c in chunks for p in lay.chunk_phys_ids(c)]
         idx = torch.tensor(ids, dtype=torch.int32, device="cuda").expand(
             w.B, w.H, L.nQB, len(ids)).contiguous()
         cnt = torch.full((w.B, w.H, L.nQB), len(ids), dtype=torch.int32, device="cuda")
@@ -508,8 +504,8 @@ def bench_dense_comparators(torch, runner, flush, reps=10):
                                 L.o, L.lse)
         fn()
         ms = _timed(torch, fn, reps, flush)
-        lens = np.array(w.chunk_block_lens(), dtype=np.int64)
-        fl = 4 * int(lens.sum()) * int(np.array([w.chunk_block_lens()[i % w.nb_c] for i in range(len(ids))]).sum()) * w.D * w.B * w.H
+        lens = np.array(lay.block_lens(), dtype=np.int64)
+        fl = 4 * int(lens.sum()) * int(lens.sum()) * len(chunks) * w.D * w.B * w.H
         out[name] = {"blocks": len(ids), "ms": round(ms, 4), "tflops": round(fl / ms / 1e9, 1)}
     return out
 
@@ -571,7 +567,7 @@ def bench_rollouts(torch, timed_steps=6):
         torch.cuda.synchronize()
         ms = float(np.mean([a.elapsed_time(b) for a, b in times]))
         kv = sum(layer_bytes(L) for L in layers)
-        dense_kv = w.n_chunks * w.nb_c * w.bs * w.D * 2 * 2 * w.B * w.H * w.layers
+        dense_kv = w.n_chunks * layers[0].layout.nb_c * w.bs * w.D * 2 * 2 * w.B * w.H * w.layers
         out[name] = {"layers": w.layers, "P": w.P, "policy": "merge_mean" if w.policy else "evict",
                      "per_chunk_ms": round(ms, 4), "timed_steps": f"{warm}..{steps - 1}",
                      "kv_bytes": kv, "dense_full_cache_kv_bytes_at_last_step": dense_kv,
@@ -625,8 +621,7 @@ def bench_hbm_at_scale(torch, flush, pk, reps=5):
         t.copy_(torch.randn(t.shape, generator=g, device="cuda").bfloat16())
     for c in range(wv.n_chunks):
         L.set_chunk_meta(c)
-    L.score(wv.n_chunks - 1, pool_ids=L.ids(("all",), [p for c in range(wv.n_chunks)
-                                                       for p in wv.chunk_phys_ids(c)]))
+    L.score(wv.n_chunks - 1, pool_ids=L.all_ids())
     ci, cs = L.candidates(wv.n_chunks - 1)
 
     L.reset_memory()
@@ -684,8 +679,8 @@ def bench_append(torch, runner, pk, reps=20):
     out = {}
     # decode chunk: 29 MB of inputs fit L2, so the graph flushes it first (as the step does)
     ms = _graph_timed(torch, lambda: L.append(t, k, v), reps, pre=flush.zero_)
-    out["append_chunk, decode chunk"] = entry(append_traffic(w.B * w.H, w.chunk_tokens, w.nb_c, w.bs,
-                                                      w.D), ms)
+    out["append_chunk, decode chunk"] = entry(append_traffic(w.B * w.H, w.chunk_tokens,
+                                                             L.layout.nb_c, w.bs, w.D), ms)
     out["score_blocks, keys pooled by the append (queries only)"] = {
         "ms": round(_graph_timed(torch, lambda: L.score(t, pool_ids=L.no_ids), reps,
                                  pre=flush.zero_), 5)}
@@ -697,39 +692,34 @@ def bench_append(torch, runner, pk, reps=20):
 
 
 # ----------------------------------------------------------------- CPU oracle
-def cpu_oracle_sample(w, snap, n_heads=2, n_qblocks=None):
-    """Time the oracle on a bounded sample: the full score/update/select on the
-    sampled heads plus attention on their query blocks.  Returns
-    (attended FLOPs of the sample, seconds, description)."""
+def cpu_oracle_sample(w, chunks, n_heads=2, n_qblocks=None):
+    """Time the oracle on a bounded sample of the decode step: its own layer
+    state for the sampled heads (every chunk written through its own
+    placement), the full score/update/select, and attention on their first
+    query blocks.  Returns (attended FLOPs of the sample, seconds,
+    description)."""
     import oracle as O
     import pbsa_inputs as PI
     H = n_heads
-    sub = {k: (v[:, :H] if isinstance(v, np.ndarray) and v.ndim >= 3 and v.shape[1] == w.H else v)
-           for k, v in snap.items()}
-    ws = PI.variant(w, H=H)
+    orc = O.OracleLayer.of(PI.variant(w, H=H))
+    for t, (_, k, v) in chunks.items():
+        orc.write_chunk(t, k[:, :H], v[:, :H])
+    t_cur = w.n_chunks - 1
+    q = chunks[t_cur][0][:, :H]
+    all_ids = [p for c in range(w.n_chunks) for p in orc.place.chunk_ids(c)]
     t0 = time.perf_counter()
-    kp = sub["kpool"].astype(np.float64)
-    vp = sub["vpool"].astype(np.float64)
-    kb0 = np.zeros((w.B, H, w.NB_phys, w.D))
-    qb, kb, S, m = O.score_blocks(sub["q"], kp, sub["blk_len"], sub["all_ids"], kb0, w.scale, w.bs)
-    up = O.update_memory(kp, vp, sub["blk_len"], sub["blk_pos"], kb, sub["slot_src"],
-                         sub["slot_w"], sub["cand_ids"], sub["cand_src"], m, w.P, w.n_sink,
-                         w.policy, w.dtype)
-    kp2, vp2, bl2, bp2 = up[0], up[1], up[2], up[3]
-    A = O.select_local(S, sub["win_ids"], w.k, PI.mem_ids_all_slots(ws), bl2, w.mask,
-                       sub["q_pos0"], bp2, w.bs, w.chunk_tokens)
-    idx, cnt = O.lists_to_arrays(A, PI.amax(w))
+    res = orc.step(t_cur, q, pool_ids=all_ids, attend=False)
+    idx, cnt = res["idx"], res["cnt"]
     nq = idx.shape[2] if n_qblocks is None else n_qblocks
-    q = sub["q"][:, :, :nq * w.bs]
-    O.attention_fwd(q, kp2, vp2, bl2, bp2, idx[:, :, :nq], cnt[:, :, :nq], w.scale, w.mask,
-                    sub["q_pos0"])
+    lens = np.array([n for _, n in orc.place.blocks], dtype=np.int64)
+    O.attention_fwd(q[:, :, :int(lens[:nq].sum())], orc.kp, orc.vp, orc.bl, orc.bp,
+                    idx[:, :, :nq], cnt[:, :, :nq], orc.scale, w.mask, t_cur * w.chunk_tokens)
     dt = time.perf_counter() - t0
-    lens = np.array(w.chunk_block_lens(), dtype=np.int64)
     fl = 0
     for h in range(H):
         for i in range(nq):
             ids = idx[0, h, i, :cnt[0, h, i]]
-            fl += 4 * int(lens[i]) * int(bl2[0, h, ids].astype(np.int64).sum()) * w.D
+            fl += 4 * int(lens[i]) * int(orc.bl[0, h, ids].astype(np.int64).sum()) * w.D
     return fl, dt, f"{H} of {w.H} heads, {nq} of {idx.shape[2]} query blocks, full score/update/select"
 
 
@@ -741,9 +731,10 @@ def cores_used():
 
 
 def config_of(w):
+    nb_c = -(-w.chunk_tokens // w.bs)
     return {"workload": (f"decode step: B{w.B} H{w.H} D{w.D} bf16, {w.bs}-token blocks, "
-                         f"query chunk {w.chunk_tokens} tokens ({w.nb_c} blocks), cache "
-                         f"{w.n_chunks} chunks ({w.n_chunks * w.nb_c} blocks), P{w.P} "
+                         f"query chunk {w.chunk_tokens} tokens ({nb_c} blocks), cache "
+                         f"{w.n_chunks} chunks ({w.n_chunks * nb_c} blocks), P{w.P} "
                          f"W{w.W} chunks k{w.k}, evict"),
             "global_batch": w.B, "seq_len": w.chunk_tokens,
             "cache_tokens": w.n_chunks * w.chunk_tokens,
@@ -876,7 +867,7 @@ def main():
         extras["append_chunk"] = bench_append(torch, runner, pk)
         line["extras"] = extras
     if rank == 0 and not args.no_cpu:
-        fl, dt, desc = cpu_oracle_sample(w, runner.snap)
+        fl, dt, desc = cpu_oracle_sample(w, runner.chunks)
         line["cpu_baseline"] = {"value": round(fl / dt / 1e12, 6), "unit": "TFLOP/s",
                                 "cores": cores_used(), "kind": "oracle", "sample": desc,
                                 "seconds": round(dt, 2)}
@@ -904,7 +895,7 @@ def run_train(args):
     T.set_meta()
     T.lists()
     torch.cuda.synchronize()
-    lens = np.array([n for c in range(w.n_chunks) for n in w.chunk_block_lens()], dtype=np.int64)
+    lens = np.array([n for c in range(w.n_chunks) for n in T.layout.block_lens()], dtype=np.int64)
     ffl = _pair_flops(T.idx.cpu().numpy(), T.cnt.cpu().numpy(), T.blk_len.cpu().numpy(), lens,
                       w.D, 4)
     flops = ffl * (4 + 10) // 4
@@ -976,13 +967,13 @@ def run_reference(args):
         return
     import pbsa_inputs as PI
     w = PI.WORKLOADS["decode"]
-    snap = PI.snapshot(w)
+    chunks = PI.snapshot_chunks(w)
     times, fls = [], []
     desc = ""
     # keep the whole run to a few minutes: smaller samples when many steps are asked
     nq = 8 if args.warmup + args.steps <= 100 else 1
     for it in range(args.warmup + args.steps):
-        fl, dt, desc = cpu_oracle_sample(w, snap, n_heads=1, n_qblocks=nq)
+        fl, dt, desc = cpu_oracle_sample(w, chunks, n_heads=1, n_qblocks=nq)
         if it >= args.warmup:
             times.append(dt)
             fls.append(fl)

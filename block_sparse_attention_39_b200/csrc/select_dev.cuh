@@ -86,6 +86,8 @@ __device__ __forceinline__ void select_row(const SelArgs& a, int i, long bh) {
 #pragma unroll
   for (int r = 0; r < U; ++r) {
     const int m = mid[r];
+    // -1 names no block; any other id outside the pool is an argument error
+    if (m >= NB || m < -1) report_status(status, PBSA_ERR_ARG);
     mlen[r] = (m >= 0 && m < NB) ? blk_len[bh * NB + m] : 0;
   }
   // ---- Top-K over the window (element order is irrelevant before the sort)
@@ -147,7 +149,12 @@ __device__ __forceinline__ void select_row(const SelArgs& a, int i, long bh) {
   int pos = incl - mine;
   int32_t* out = idx + (bh * nQB_total + qb_offset + i) * static_cast<long>(Amax);
   if (total > Amax) {
+    // the list does not fit: report it and leave an empty, defined list so
+    // that a later attention call on the same stream attends nothing rather
+    // than a previous call's blocks
     if (lane == 0) report_status(status, PBSA_ERR_SHAPE);
+    for (int e = lane; e < Amax; e += 32) out[e] = -1;
+    if (lane == 0) cnt[bh * nQB_total + qb_offset + i] = 0;
     return;
   }
 #pragma unroll

@@ -9,12 +9,12 @@ calls into the C ABI; the host side only decides which physical ids are passed
 """
 from __future__ import annotations
 
-from typing import Optional
+import math
 
 import torch
 
 from . import pbsa as K
-from pbsa_inputs import Workload
+from .layout import PoolLayout
 
 
 def _i32(x, device):
@@ -22,17 +22,24 @@ def _i32(x, device):
 
 
 class PbsaLayer:
-    def __init__(self, w: Workload, device="cuda", P_override: Optional[int] = None):
-        self.w = w
+    """cfg: any object with the layer's shape as attributes -- B, H, D, bs,
+    dtype ("bf16" / "f32"), chunk_tokens, P, n_sink, W, k, policy, mask,
+    n_chunks (resident chunks of a snapshot, or the rollout's length) and
+    rollout (ring of W + 1 chunk positions)."""
+
+    def __init__(self, cfg, device="cuda"):
+        self.w = w = cfg
+        self.layout = lay = PoolLayout.of(cfg)
         self.dev = torch.device(device)
         B, H, D, bs = w.B, w.H, w.D, w.bs
+        self.scale = 1.0 / math.sqrt(D)
         self.tdtype = torch.bfloat16 if w.dtype == "bf16" else torch.float32
-        self.d = K.dims(B, H, D, bs, w.scale, self.tdtype)
-        self.dbf = K.dims(B, H, D, bs, w.scale, torch.bfloat16)
-        self.P = w.n_slots
-        self.NB = w.NB_phys
-        self.nQB = w.nb_c
-        self.Amax = self.P + w.k if w.slots_in_pool else w.P + w.k
+        self.d = K.dims(B, H, D, bs, self.scale, self.tdtype)
+        self.dbf = K.dims(B, H, D, bs, self.scale, torch.bfloat16)
+        self.P = lay.P
+        self.NB = lay.NB
+        self.nQB = lay.nb_c
+        self.Amax = self.P + w.k
         NB, P = self.NB, self.P
         dev = self.dev
         self.kpool = torch.zeros(B, H, NB, bs, D, dtype=self.tdtype, device=dev)
@@ -51,7 +58,7 @@ class PbsaLayer:
         self.o = torch.zeros(B, H, w.chunk_tokens, D, dtype=torch.bfloat16, device=dev)
         self.lse = torch.zeros(B, H, w.chunk_tokens, dtype=torch.float32, device=dev)
         self.mem_ids = _i32(torch.arange(P).expand(B, H, P), dev) if P else None
-        max_cand = w.nb_c * (len(w.snapshot_candidate_chunks()) if not w.rollout else 1)
+        max_cand = lay.nb_c * (len(lay.older_chunks(w.n_chunks - 1)) if not w.rollout else 1)
         self.max_cand = max(max_cand, 1)
         ws = K.update_memory_workspace(self.d, max(P, 1), self.max_cand)
         self.ws = torch.empty(ws, dtype=torch.uint8, device=dev)
@@ -76,13 +83,18 @@ class PbsaLayer:
         return t
 
     def chunk_ids(self, t):
-        return self.ids(("chunk", t % self.w.ring_chunks if self.w.rollout else t),
-                        self.w.chunk_phys_ids(t))
+        return self.ids(("chunk", self.layout.position(t)), self.layout.chunk_phys_ids(t))
 
     def window_ids(self, t):
-        chunks = self.w.window_chunks(t)
-        key = ("win",) + tuple(c % self.w.ring_chunks if self.w.rollout else c for c in chunks)
-        return self.ids(key, [p for c in chunks for p in self.w.chunk_phys_ids(c)])
+        lay = self.layout
+        chunks = lay.window_chunks(t)
+        key = ("win",) + tuple(lay.position(c) for c in chunks)
+        return self.ids(key, [p for c in chunks for p in lay.chunk_phys_ids(c)])
+
+    def all_ids(self):
+        """Every resident chunk block (a snapshot's cache)."""
+        lay = self.layout
+        return self.ids(("all",), [p for c in range(lay.positions) for p in lay.chunk_phys_ids(c)])
 
     # ------------------------------------------------------------ state
     def reset_memory(self):
@@ -96,16 +108,16 @@ class PbsaLayer:
 
     def set_chunk_meta(self, t):
         """Lengths and positions of chunk t's blocks (where the ring puts them)."""
-        lens = self.w.chunk_block_lens()
-        for j, pid in enumerate(self.w.chunk_phys_ids(t)):
-            self.blk_len[:, :, pid] = lens[j]
-            self.blk_pos[:, :, pid] = t * self.w.chunk_tokens + j * self.w.bs
+        lay = self.layout
+        for j, (pid, n) in enumerate(zip(lay.chunk_phys_ids(t), lay.block_lens())):
+            self.blk_len[:, :, pid] = n
+            self.blk_pos[:, :, pid] = t * lay.chunk_tokens + j * lay.bs
 
     def write_chunk(self, t, k_chunk, v_chunk):
         """Place a chunk's K/V [B,H,T_c,D] into its blocks (the caller's cache append)."""
         w = self.w
-        ids = w.chunk_phys_ids(t)
-        lens = w.chunk_block_lens()
+        ids = self.layout.chunk_phys_ids(t)
+        lens = self.layout.block_lens()
         for j, pid in enumerate(ids):
             r0 = j * w.bs
             self.kpool[:, :, pid, :lens[j]] = k_chunk[:, :, r0:r0 + lens[j]]
@@ -161,15 +173,15 @@ class PbsaLayer:
     def candidates(self, t):
         """Blocks that leave the window when chunk t arrives (rollout) or every
         block older than the window (snapshot)."""
-        w = self.w
-        if w.rollout:
-            c = w.leaving_chunk(t)
+        lay = self.layout
+        if lay.rollout:
+            c = lay.leaving_chunk(t)
             chunks = [] if c is None else [c]
         else:
-            chunks = w.snapshot_candidate_chunks()
-        key = ("cand",) + tuple(chunks) if not w.rollout else ("cand", t)
-        ci = self.ids(key + ("phys",), [p for c in chunks for p in w.chunk_phys_ids(c)])
-        cs = self.ids(key + ("src",), [g for c in chunks for g in w.chunk_global_ids(c)])
+            chunks = lay.older_chunks(t)
+        key = ("cand",) + tuple(chunks) if not lay.rollout else ("cand", t)
+        ci = self.ids(key + ("phys",), [p for c in chunks for p in lay.chunk_phys_ids(c)])
+        cs = self.ids(key + ("src",), [g for c in chunks for g in lay.chunk_global_ids(c)])
         return ci, cs
 
     def route(self, t, stream=None, appended=False):
@@ -220,18 +232,21 @@ class PbsaTrain:
     sweep, the top ceil(d * allowed) of all allowed blocks per query block
     (``lists(density=d)``)."""
 
-    def __init__(self, w: Workload, device="cuda"):
-        assert not w.slots_in_pool
-        self.w = w
+    def __init__(self, cfg, device="cuda"):
+        self.w = w = cfg
+        self.layout = lay = PoolLayout(w.chunk_tokens, w.bs, 0, w.W, w.n_chunks, rollout=False,
+                                       slots_in_pool=False)
         dev = torch.device(device)
         self.dev = dev
         B, H, D, bs = w.B, w.H, w.D, w.bs
+        self.scale = 1.0 / math.sqrt(D)
         self.T = w.n_chunks * w.chunk_tokens
         self.G = w.n_chunks
-        self.nQB = w.n_chunks * w.nb_c
-        self.NB = w.NB_phys
-        self.d = K.dims(B, H, D, bs, w.scale, torch.bfloat16, q_chunk=w.chunk_tokens)
-        self.d1 = K.dims(B, H, D, bs, w.scale, torch.bfloat16)
+        self.nb_c = lay.nb_c
+        self.nQB = w.n_chunks * lay.nb_c
+        self.NB = lay.NB
+        self.d = K.dims(B, H, D, bs, self.scale, torch.bfloat16, q_chunk=w.chunk_tokens)
+        self.d1 = K.dims(B, H, D, bs, self.scale, torch.bfloat16)
         self.q = torch.zeros(B, H, self.T, D, dtype=torch.bfloat16, device=dev)
         self.kpool = torch.zeros(B, H, self.NB, bs, D, dtype=torch.bfloat16, device=dev)
         self.vpool = torch.zeros_like(self.kpool)
@@ -265,39 +280,49 @@ class PbsaTrain:
         return t
 
     def set_meta(self):
-        w = self.w
-        lens = w.chunk_block_lens()
-        for t in range(w.n_chunks):
-            for j, pid in enumerate(w.chunk_phys_ids(t)):
-                self.blk_len[:, :, pid] = lens[j]
-                self.blk_pos[:, :, pid] = t * w.chunk_tokens + j * w.bs
+        lay = self.layout
+        for t in range(self.G):
+            for j, (pid, n) in enumerate(zip(lay.chunk_phys_ids(t), lay.block_lens())):
+                self.blk_len[:, :, pid] = n
+                self.blk_pos[:, :, pid] = t * lay.chunk_tokens + j * lay.bs
+
+    def write_chunk(self, t, k_chunk, v_chunk):
+        """Chunk t's K/V [B,H,T_c,D] into its blocks (padding rows zero)."""
+        lay = self.layout
+        for j, (pid, n) in enumerate(zip(lay.chunk_phys_ids(t), lay.block_lens())):
+            r0 = j * lay.bs
+            self.kpool[:, :, pid].zero_()
+            self.vpool[:, :, pid].zero_()
+            self.kpool[:, :, pid, :n] = k_chunk[:, :, r0:r0 + n]
+            self.vpool[:, :, pid, :n] = v_chunk[:, :, r0:r0 + n]
 
     def lists(self, density=None, stream=None):
-        w = self.w
+        w, lay = self.w, self.layout
+        nb_c = lay.nb_c
         K.score_blocks(self.d, self.q, self.T, self.kpool, self.NB, self.blk_len, self.all_ids,
                        self.NB, self.q_bar, self.k_bar, self.scores, self.mem, stream)
         for t in range(self.G):
             if density is None:
-                older = [p for c in range(0, max(0, t - w.W + 1)) for p in w.chunk_phys_ids(c)]
+                older = [p for c in lay.older_chunks(t) for p in lay.chunk_phys_ids(c)]
                 if older:
                     o_ids = self.ids(("older", t), older)
                     K.select_local(self.d1, self.mem, 1, self.NB, o_ids, len(older), w.P, None, 0,
                                    self.blk_len, 0, 0, None, w.bs, self.mem_idx, self.mem_cnt,
                                    w.P, t, self.G, stream)
-                win = self.ids(("win", t), [p for c in w.window_chunks(t)
-                                            for p in w.chunk_phys_ids(c)])
-                K.select_local(self.d1, self.scores, w.nb_c, self.NB, win, win.numel(), w.k,
+                win = self.ids(("win", t), [p for c in lay.window_chunks(t)
+                                            for p in lay.chunk_phys_ids(c)])
+                K.select_local(self.d1, self.scores, nb_c, self.NB, win, win.numel(), w.k,
                                self.mem_idx, w.P, self.blk_len, 0, t * w.chunk_tokens,
                                self.blk_pos, w.chunk_tokens, self.idx, self.cnt, self.Amax,
-                               t * w.nb_c, self.nQB, stream, mem_ld=self.G * w.P,
+                               t * nb_c, self.nQB, stream, mem_ld=self.G * w.P,
                                mem_offset=t * w.P)
             else:
-                allowed = [p for c in range(t + 1) for p in w.chunk_phys_ids(c)]
+                allowed = [p for c in range(t + 1) for p in lay.chunk_phys_ids(c)]
                 kd = max(1, int(-(-density * len(allowed) // 1)))
                 a_ids = self.ids(("allowed", t), allowed)
-                K.select_local(self.d1, self.scores, w.nb_c, self.NB, a_ids, len(allowed), kd,
+                K.select_local(self.d1, self.scores, nb_c, self.NB, a_ids, len(allowed), kd,
                                None, 0, self.blk_len, 0, t * w.chunk_tokens, self.blk_pos,
-                               w.chunk_tokens, self.idx, self.cnt, self.Amax, t * w.nb_c,
+                               w.chunk_tokens, self.idx, self.cnt, self.Amax, t * nb_c,
                                self.nQB, stream)
 
     def fwd(self, stream=None):

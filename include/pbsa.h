@@ -13,8 +13,11 @@
  * Conventions shared by every call
  * --------------------------------
  *  - All tensor arguments are DEVICE pointers owned by the caller; the library
- *    allocates no device memory.  The only library-owned device state is one
- *    status word per device (a __device__ variable, see pbsa_get_status).
+ *    allocates no device memory at run time.  Its device state is static,
+ *    created when the library is loaded on a device: one status word per
+ *    device (a __device__ variable, see pbsa_get_status) and the 16 MiB
+ *    scratch array of pbsa_attn_bwd_noalloc (a __device__ array that every
+ *    device which loads the library holds until the process exits).
  *  - `stream` is a cudaStream_t passed as void*.  Every call is asynchronous
  *    on that stream; nothing synchronises except pbsa_get_status.
  *  - Batch-major layouts, all contiguous:
@@ -187,6 +190,12 @@ int pbsa_update_memory(const pbsa_dims* dims, void* kpool, void* vpool, int NB,
  *                with local, ascending, without duplicates.
  * Written to idx[b,h,r,0..cnt) (rest -1) and cnt[b,h,r].
  *
+ * Errors found on the device: a list longer than Amax sets PBSA_ERR_SHAPE and
+ * writes an empty row (cnt 0, every entry -1), so a later attention call on
+ * the same stream attends nothing for that row rather than stale blocks; a
+ * win_ids entry outside [0, NB), or a mem_ids entry outside [-1, NB), sets
+ * PBSA_ERR_ARG and is skipped.
+ *
  * scores: [B,H,nQB_total,NB] float, indexed by the same physical ids as
  * blk_len and blk_pos [B,H,NB].  win_ids: device int32 [n_win], same for every
  * (b,h).  mem_ids: device int32, row (b,h) at mem_ids + (b*H+h)*mem_ld
@@ -335,8 +344,10 @@ int pbsa_attn_bwd(const pbsa_dims* dims, const void* q, int Tq, int q_pos0,
  * cudaFree, no allocating library routine.
  *
  * The first call on a device looks up the array's device address (once per
- * device, with that device current); make that first call before any stream
- * capture.  All calls share the one array, which keeps the previous call's
+ * device, with that device current) and caches it for the life of the
+ * process; make that first call before any stream capture.  cudaDeviceReset
+ * invalidates the cached address: do not call this entry point on a device
+ * after resetting it.  All calls share the one array, which keeps the previous call's
  * contents (each call clears what must start at zero): calls that may overlap
  * on the GPU -- different streams, or different host threads -- race on it
  * and must be ordered by the caller.

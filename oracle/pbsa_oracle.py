@@ -74,17 +74,33 @@ def round_storage(x: np.ndarray, dtype: str) -> np.ndarray:
 # a1  block compression by pooling
 # ---------------------------------------------------------------------------
 
+def chunk_blocks(T_c: int, bs: int):
+    """The blocks one chunk of T_c token rows is cut into (R9): runs of bs
+    consecutive rows from the chunk's first row, the last run shorter when bs
+    does not divide T_c.  Returns (first row within the chunk, length) per
+    block.  Key chunks and query chunks are tiled alike; a 4680-token chunk in
+    128-token blocks gives 36 full blocks and one of 72 rows."""
+    out = []
+    r0 = 0
+    while r0 < T_c:
+        n = min(bs, T_c - r0)
+        out.append((r0, n))
+        r0 += n
+    return out
+
+
 def query_blocks(Tq: int, bs: int, q_chunk: int = 0):
     """Query rows are a sequence of chunks of q_chunk rows (0: one chunk of Tq
     rows; the last chunk may be shorter), and each chunk is tiled into blocks
-    of bs rows on its own, its last block partial (R9).  Returns the list of
-    (first row, length) of every query block."""
+    on its own by ``chunk_blocks`` (R9), so no block crosses a chunk boundary.
+    Returns the list of (first row, length) of every query block."""
     qc = q_chunk if q_chunk > 0 else Tq
     out = []
-    for c0 in range(0, Tq, qc):
+    c0 = 0
+    while c0 < Tq:
         clen = min(qc, Tq - c0)
-        for b0 in range(0, clen, bs):
-            out.append((c0 + b0, min(bs, clen - b0)))
+        out.extend((c0 + r0, n) for r0, n in chunk_blocks(clen, bs))
+        c0 += clen
     return out
 
 
@@ -491,3 +507,206 @@ def attention_bwd(q, kpool, vpool, blk_len, blk_pos, idx, cnt, dO, scale: float,
                     dv[b, h, j, :m] += dvc[off:off + m]
                     off += m
     return dq, dk, dv
+
+
+# ---------------------------------------------------------------------------
+# the chunk step: the local window, the blocks leaving it, and where blocks sit
+# ---------------------------------------------------------------------------
+
+def window_chunks(t: int, W: int):
+    """The chunks of the local window L_t while chunk t is generated (R7): the
+    W most recent chunks, chunk t itself included; fewer while the rollout is
+    shorter than W chunks (Sparse Forcing, gist.science/es, section 2
+    "Arquitectura Propuesta", item "Ventana Local")."""
+    return [c for c in range(t - W + 1, t + 1) if c >= 0]
+
+
+def leaving_chunk(t: int, W: int):
+    """The chunk that drops out of the local window when chunk t arrives (R14):
+    the chunk of L_{t-1} that is not in L_t, or None while the window is still
+    filling.  Its blocks are the new candidates of the memory update
+    (section 2 "Arquitectura Propuesta", item "Mecanismo de Actualización":
+    Top-C retention over the blocks that leave the local window)."""
+    if t == 0:
+        return None
+    gone = set(window_chunks(t - 1, W)) - set(window_chunks(t, W))
+    assert len(gone) <= 1
+    return gone.pop() if gone else None
+
+
+def older_chunks(t: int, W: int):
+    """Every chunk before chunk t that is not in its window L_t: the chunks a
+    snapshot step offers to the persistent memory, and the chunks the
+    trainable path's persistent set is chosen from (R13)."""
+    win = set(window_chunks(t, W))
+    return [c for c in range(t) if c not in win]
+
+
+class PoolPlacement:
+    """Physical ids of the blocks in the pool of one (b, h).
+
+    The library addresses blocks by physical id in a pool [NB, bs, D] per
+    (b, h).  The convention below is the one the tests and the engine both
+    follow (each side writes it on its own):
+
+    * ids [0, P) are the persistent slots (P = 0: no slots);
+    * then positions of nb_c ids each, one chunk per position: chunk t at
+      position t when every chunk stays resident (snapshot), or at position
+      t mod (W + 1) in a rollout, whose ring is one chunk longer than the
+      window so that the chunk leaving the window is still readable while the
+      memory update of the step consumes it (R14);
+    * block j of chunk t has the global (source) id t * nb_c + j.
+    """
+
+    def __init__(self, P: int, T_c: int, bs: int, W: int, n_chunks: int, ring: bool):
+        self.P = P
+        self.blocks = chunk_blocks(T_c, bs)
+        self.nb_c = len(self.blocks)
+        self.positions = W + 1 if ring else n_chunks
+        self.ring = ring
+        self.NB = P + self.positions * self.nb_c
+
+    def chunk_ids(self, t: int):
+        pos = t % self.positions if self.ring else t
+        assert 0 <= pos < self.positions
+        first = self.P + pos * self.nb_c
+        return [first + j for j in range(self.nb_c)]
+
+    def global_ids(self, t: int):
+        return [t * self.nb_c + j for j in range(self.nb_c)]
+
+
+class OracleLayer:
+    """The oracle's state of one attention layer, advanced chunk by chunk.
+
+    One step of chunk t follows the order taken in R14: the chunk's keys and
+    values are written into their blocks, then the blocks are scored, the
+    persistent memory is updated with the blocks that leave the window as new
+    candidates (a snapshot step offers every chunk older than the window to an
+    empty memory), the local Top-K is selected and the chunk's queries attend
+    the union of the memory and their local blocks.  Attention takes bf16
+    inputs (R17: an fp32 cache is attended through bf16 copies)."""
+
+    def __init__(self, B, H, D, bs, T_c, P, n_sink, W, k, policy, mask, store, n_chunks,
+                 ring):
+        self.B, self.H, self.D, self.bs, self.T_c = B, H, D, bs, T_c
+        self.P, self.n_sink, self.W, self.k = P, n_sink, W, k
+        self.policy, self.mask, self.store, self.ring = policy, mask, store, ring
+        self.scale = 1.0 / math.sqrt(D)
+        self.place = PoolPlacement(P, T_c, bs, W, n_chunks, ring)
+        NB = self.place.NB
+        self.kp = np.zeros((B, H, NB, bs, D))
+        self.vp = np.zeros_like(self.kp)
+        self.bl = np.zeros((B, H, NB), dtype=np.int32)
+        self.bp = np.zeros((B, H, NB), dtype=np.int32)
+        self.kb = np.zeros((B, H, NB, D))
+        self.ss = np.full((B, H, P), -1, dtype=np.int64)
+        self.sw = np.zeros((B, H, P))
+
+    @classmethod
+    def of(cls, w):
+        """Build from any object carrying the layer's shape as attributes."""
+        return cls(w.B, w.H, w.D, w.bs, w.chunk_tokens, w.P if w.slots_in_pool else 0,
+                   w.n_sink, w.W, w.k, w.policy, w.mask, w.dtype, w.n_chunks, w.rollout)
+
+    @property
+    def Amax(self):
+        return self.P + self.k
+
+    def write_chunk(self, t, k, v):
+        """Chunk t's keys and values [B,H,T_c,D] into its blocks; padding rows are zero."""
+        for pid, (r0, n) in zip(self.place.chunk_ids(t), self.place.blocks):
+            self.kp[:, :, pid] = 0.0
+            self.vp[:, :, pid] = 0.0
+            self.kp[:, :, pid, :n] = k[:, :, r0:r0 + n]
+            self.vp[:, :, pid, :n] = v[:, :, r0:r0 + n]
+            self.bl[:, :, pid] = n
+            self.bp[:, :, pid] = t * self.T_c + r0
+
+    def window_ids(self, t):
+        return [p for c in window_chunks(t, self.W) for p in self.place.chunk_ids(c)]
+
+    def candidates(self, t):
+        """(physical ids, global ids) offered to the memory at step t."""
+        if self.ring:
+            c = leaving_chunk(t, self.W)
+            chunks = [] if c is None else [c]
+        else:
+            chunks = older_chunks(t, self.W)
+        return ([p for c in chunks for p in self.place.chunk_ids(c)],
+                [g for c in chunks for g in self.place.global_ids(c)])
+
+    def step(self, t, q, pool_ids=None, attend=True):
+        """Score -> update -> select -> attend for chunk t (already written).
+
+        pool_ids: the blocks whose pooled keys are (re)computed (default: the
+        chunk's own blocks; older pooled keys are kept).  Returns every
+        intermediate result."""
+        ids = self.place.chunk_ids(t) if pool_ids is None else list(pool_ids)
+        q_bar, self.kb, S, m = score_blocks(q, self.kp, self.bl, ids, self.kb, self.scale,
+                                            self.bs)
+        pre_kb = self.kb.copy()
+        ci, cs = self.candidates(t)
+        info = None
+        if self.P and ci:
+            out = update_memory(self.kp, self.vp, self.bl, self.bp, self.kb, self.ss, self.sw,
+                                ci, cs, m, self.P, self.n_sink, self.policy, self.store)
+            self.kp, self.vp, self.bl, self.bp, self.kb, self.ss, self.sw, info = out
+        mem = (np.broadcast_to(np.arange(self.P), (self.B, self.H, self.P))
+               if self.P else None)
+        A = select_local(S, self.window_ids(t), self.k, mem, self.bl, self.mask,
+                         t * self.T_c, self.bp, self.bs, self.T_c)
+        idx, cnt = lists_to_arrays(A, self.Amax)
+        res = dict(q_bar=q_bar, k_bar=pre_kb, S=S, m=m, info=info, A=A, idx=idx, cnt=cnt,
+                   cand_ids=ci, cand_src=cs, win_ids=self.window_ids(t), kpool=self.kp,
+                   vpool=self.vp, blk_len=self.bl, blk_pos=self.bp, k_bar2=self.kb,
+                   slot_src=self.ss, slot_w=self.sw)
+        if attend:
+            q16, k16, v16 = round_bf16(q), round_bf16(self.kp), round_bf16(self.vp)
+            res["O"], res["lse"] = attention_fwd(q16, k16, v16, self.bl, self.bp, idx, cnt,
+                                                 self.scale, self.mask, t * self.T_c)
+            res.update(q16=q16, k16=k16, v16=v16)
+        return res
+
+
+def trainable_lists(q, kpool, blk_len, T_c, bs, P, W, k, scale, density=None):
+    """Attended lists of the trainable path over a whole sequence of chunks
+    (R13): no slots; chunk t's blocks sit at ids t*nb_c .. (t+1)*nb_c - 1 and
+    selection is one-shot per query chunk t:
+
+    * density None: the persistent set is the top-P blocks of the chunks older
+      than the window by chunk t's memory score, united with the top-k window
+      blocks of each query block by block score (the inference rule applied
+      with an empty memory refilled for every chunk);
+    * density d (R18): the top ceil(d * n) blocks by block score of the n
+      chunk-causally allowed blocks (every block of chunks 0..t).
+
+    q: [B,H,n_chunks*T_c,D]; kpool [B,H,n_chunks*nb_c,bs,D].  Returns
+    (idx, cnt) with Amax = P + k (density None) or all blocks."""
+    B, H = q.shape[:2]
+    n_chunks = q.shape[2] // T_c
+    place = PoolPlacement(0, T_c, bs, W, n_chunks, ring=False)
+    NB = place.NB
+    kb = pool_keys(kpool, blk_len, range(NB), np.zeros((B, H, NB, q.shape[3])))
+    nb_c = place.nb_c
+    A = [[[None] * (n_chunks * nb_c) for _ in range(H)] for _ in range(B)]
+    for t in range(n_chunks):
+        S = block_scores(pool_queries(q[:, :, t * T_c:(t + 1) * T_c], bs), kb, scale)
+        if density is None:
+            older = [p for c in older_chunks(t, W) for p in place.chunk_ids(c)]
+            mem_ids = np.full((B, H, P), -1, dtype=np.int64)
+            if older:
+                chosen = select_local(memory_scores(S)[:, :, None, :], older, P, None, blk_len)
+                for b in range(B):
+                    for h in range(H):
+                        mem_ids[b, h, :len(chosen[b][h][0])] = chosen[b][h][0]
+            win = [p for c in window_chunks(t, W) for p in place.chunk_ids(c)]
+            At = select_local(S, win, k, mem_ids, blk_len)
+        else:
+            allowed = [p for c in range(t + 1) for p in place.chunk_ids(c)]
+            At = select_local(S, allowed, int(math.ceil(density * len(allowed))), None, blk_len)
+        for b in range(B):
+            for h in range(H):
+                for i in range(nb_c):
+                    A[b][h][t * nb_c + i] = At[b][h][i]
+    return lists_to_arrays(A, P + k if density is None else NB)

@@ -2,6 +2,8 @@
 the oracle pipeline of one step, and the near-tie comparison rule."""
 from __future__ import annotations
 
+import math
+
 import numpy as np
 import torch
 
@@ -27,12 +29,18 @@ def host(t: torch.Tensor) -> np.ndarray:
         else t.detach().cpu().numpy()
 
 
-def load_layer(layer, snap, w):
-    layer.kpool.copy_(dev_storage(snap["kpool"], w.dtype))
-    layer.vpool.copy_(dev_storage(snap["vpool"], w.dtype))
-    layer.blk_len.copy_(dev_i32(snap["blk_len"]))
-    layer.blk_pos.copy_(dev_i32(snap["blk_pos"]))
-    layer.q.copy_(dev_storage(snap["q"], w.dtype))
+def snapshot_case(w):
+    """A snapshot step's inputs: every chunk of the cache as seeded tensors
+    (``{t: (q or None, k, v)}``) and the current chunk's index."""
+    return PI.snapshot_chunks(w), w.n_chunks - 1
+
+
+def load_snapshot(layer, w, chunks):
+    """The GPU side of a snapshot: every chunk written through the engine's own
+    placement, the current chunk's queries, an empty memory."""
+    for t, (_, k, v) in chunks.items():
+        layer.write_chunk(t, dev_storage(k, w.dtype), dev_storage(v, w.dtype))
+    layer.q.copy_(dev_storage(chunks[w.n_chunks - 1][0], w.dtype))
     layer.reset_memory()
 
 
@@ -52,25 +60,19 @@ def band_ok(chosen, keys: dict, n_take: int, tie=TIE):
     return (must <= chosen and not (chosen & never)), False
 
 
-def oracle_snapshot_step(w, snap):
-    """The oracle's score -> update -> select -> attend on a snapshot input."""
-    kp = snap["kpool"].astype(np.float64)
-    vp = snap["vpool"].astype(np.float64)
-    kb0 = np.zeros((w.B, w.H, w.NB_phys, w.D))
-    qb, kb, S, m = O.score_blocks(snap["q"], kp, snap["blk_len"], snap["all_ids"], kb0, w.scale,
-                                  w.bs)
-    up = O.update_memory(kp, vp, snap["blk_len"], snap["blk_pos"], kb, snap["slot_src"],
-                         snap["slot_w"], snap["cand_ids"], snap["cand_src"], m, w.P, w.n_sink,
-                         w.policy, w.dtype)
-    kp2, vp2, bl2, bp2, kb2, ss2, sw2, info = up
-    A = O.select_local(S, snap["win_ids"], w.k, PI.mem_ids_all_slots(w), bl2, w.mask,
-                       snap["q_pos0"], bp2, w.bs, w.chunk_tokens)
-    idx, cnt = O.lists_to_arrays(A, PI.amax(w))
-    q16, k16, v16 = O.round_bf16(snap["q"]), O.round_bf16(kp2), O.round_bf16(vp2)
-    out, lse = O.attention_fwd(q16, k16, v16, bl2, bp2, idx, cnt, w.scale, w.mask, snap["q_pos0"])
-    return dict(q_bar=qb, k_bar=kb, S=S, m=m, kpool=kp2, vpool=vp2, blk_len=bl2, blk_pos=bp2,
-                k_bar2=kb2, slot_src=ss2, slot_w=sw2, info=info, A=A, idx=idx, cnt=cnt, O=out,
-                lse=lse, q16=q16, k16=k16, v16=v16)
+def oracle_snapshot_step(w, chunks):
+    """The oracle's score -> update -> select -> attend on a snapshot: its own
+    layer state, every chunk written through its own placement, every
+    resident block pooled, the memory empty."""
+    orc = O.OracleLayer.of(w)
+    for t, (_, k, v) in chunks.items():
+        orc.write_chunk(t, k, v)
+    t_cur = w.n_chunks - 1
+    all_ids = [p for c in range(w.n_chunks) for p in orc.place.chunk_ids(c)]
+    ref = orc.step(t_cur, chunks[t_cur][0], pool_ids=all_ids)
+    ref.update(orc=orc, all_ids=all_ids, q_pos0=t_cur * w.chunk_tokens,
+               new_ids=orc.place.chunk_ids(t_cur))
+    return ref
 
 
 def attn_errors(o_gpu: np.ndarray, o_ref: np.ndarray, rows=None):
@@ -78,3 +80,25 @@ def attn_errors(o_gpu: np.ndarray, o_ref: np.ndarray, rows=None):
     if rows is not None:
         d = d[rows]
     return float(d.max()), float(d.mean())
+
+
+def check_step_attention(L, w, ref, q):
+    """The attention of a whole GPU step, checked without depending on near-tie
+    luck: the GPU's O and LSE against the oracle's attention over the GPU's own
+    lists and its own post-update pool (both read back), and, when the GPU's
+    lists and kept slots equal the oracle's, against the oracle's own step."""
+    idx, cnt = host(L.idx), host(L.cnt)
+    q16 = O.round_bf16(q)
+    own_o, own_l = O.attention_fwd(q16, O.round_bf16(host(L.kpool)), O.round_bf16(host(L.vpool)),
+                                   host(L.blk_len), host(L.blk_pos), idx, cnt, 1 / math.sqrt(w.D),
+                                   w.mask, ref["q_pos0"])
+    mx, mean = attn_errors(host(L.o), own_o)
+    assert mx <= ATT_MAX and mean <= ATT_MEAN, ("own lists", mx, mean)
+    np.testing.assert_allclose(host(L.lse), own_l, atol=2e-3, rtol=0)
+    same = (np.array_equal(cnt, ref["cnt"]) and np.array_equal(idx, ref["idx"]) and
+            np.array_equal(host(L.slot_src), ref["slot_src"]))
+    if same:
+        mx, mean = attn_errors(host(L.o), ref["O"])
+        assert mx <= ATT_MAX and mean <= ATT_MEAN, ("oracle step", mx, mean)
+        np.testing.assert_allclose(host(L.lse), ref["lse"], atol=2e-3, rtol=0)
+    return same

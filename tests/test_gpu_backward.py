@@ -120,109 +120,95 @@ def test_backward_chunked_query_tiling(bs, mask):
         assert ok, (name, info)
 
 
-def _train_lists(w, q, kpool, blk_len):
-    """Oracle lists of the trainable path (one-shot selection per query chunk):
-    persistent = top-P blocks older than the window by the chunk's memory score,
-    local = top-k window blocks per query block by block score."""
-    kb = O.pool_keys(kpool, blk_len, range(w.NB_phys), np.zeros((w.B, w.H, w.NB_phys, w.D)))
-    nQB = w.n_chunks * w.nb_c
-    A = [[[None] * nQB for _ in range(w.H)] for _ in range(w.B)]
-    for t in range(w.n_chunks):
-        qt = q[:, :, t * w.chunk_tokens:(t + 1) * w.chunk_tokens]
-        S = O.block_scores(O.pool_queries(qt, w.bs), kb, w.scale)
-        m = O.memory_scores(S)
-        older = [p for c in range(0, max(0, t - w.W + 1)) for p in w.chunk_phys_ids(c)]
-        mem = O.select_local(m[:, :, None, :], older, w.P, None, blk_len)
-        mem_ids = np.full((w.B, w.H, w.P), -1, dtype=np.int32)
-        for b in range(w.B):
-            for h in range(w.H):
-                mem_ids[b, h, :len(mem[b][h][0])] = mem[b][h][0]
-        win = [p for c in w.window_chunks(t) for p in w.chunk_phys_ids(c)]
-        At = O.select_local(S, win, w.k, mem_ids, blk_len)
-        for b in range(w.B):
-            for h in range(w.H):
-                for i in range(w.nb_c):
-                    A[b][h][t * w.nb_c + i] = At[b][h][i]
-    return O.lists_to_arrays(A, w.P + w.k)
+def _train_inputs(w):
+    """The trainable shape's inputs on the oracle side: the whole sequence's
+    queries and a block pool built through the oracle's own placement (no
+    slots, chunk t at ids t*nb_c ..)."""
+    chunks = [PI.chunk_tensors(w, t) for t in range(w.n_chunks)]
+    q = np.concatenate([c[0] for c in chunks], axis=2)
+    orc = O.OracleLayer(w.B, w.H, w.D, w.bs, w.chunk_tokens, 0, 0, w.W, w.k, w.policy, w.mask,
+                        w.dtype, w.n_chunks, ring=False)
+    for t, c in enumerate(chunks):
+        orc.write_chunk(t, c[1], c[2])
+    return q, orc.kp, orc.vp, orc.bl, orc.bp, chunks
 
 
 @pytest.mark.slow
-def test_backward_train_shape_sampled_heads():
+@pytest.mark.parametrize("density", [None, 0.05, 0.50])
+def test_backward_train_shape_sampled_heads(density):
+    """Forward and backward at the trainable shape's full size (B2 H12, 32 760
+    tokens, 259 blocks) with the oracle's lists: the one-shot P32 + top-16
+    lists, and the density sweep's 5 % and 50 % lists; the oracle checks two
+    sampled heads."""
     w = PI.WORKLOADS["train"]
-    chunks = [PI.chunk_tensors(w, t) for t in range(w.n_chunks)]
-    q = np.concatenate([c[0] for c in chunks], axis=2)
-    kpool = PI.pool_from_chunks(w, {t: c[1] for t, c in enumerate(chunks)})
-    vpool = PI.pool_from_chunks(w, {t: c[2] for t, c in enumerate(chunks)})
-    del chunks
-    blk_len, blk_pos = PI.chunk_layout(w, range(w.n_chunks))
+    q, kpool, vpool, blk_len, blk_pos, _ = _train_inputs(w)
+    NB = kpool.shape[2]
+    scale = 1 / math.sqrt(w.D)
     T = q.shape[2]
     dO = PI.grad_output(w, T)
-    idx, cnt = _train_lists(w, q, kpool, blk_len)
-    d = K.dims(w.B, w.H, w.D, w.bs, w.scale, torch.bfloat16, q_chunk=w.chunk_tokens)
+    idx, cnt = O.trainable_lists(q, kpool, blk_len, w.chunk_tokens, w.bs, w.P, w.W, w.k, scale,
+                                 density=density)
+    d = K.dims(w.B, w.H, w.D, w.bs, scale, torch.bfloat16, q_chunk=w.chunk_tokens)
     # forward on the GPU with the oracle's lists (O, LSE feed the backward)
     qd, kd, vd = dev_storage(q, "bf16"), dev_storage(kpool, "bf16"), dev_storage(vpool, "bf16")
     o = torch.empty(w.B, w.H, T, w.D, dtype=torch.bfloat16, device="cuda")
     lse = torch.empty(w.B, w.H, T, dtype=torch.float32, device="cuda")
-    K.attn_fwd(d, qd, T, 0, kd, vd, w.NB_phys, dev_i32(blk_len), dev_i32(blk_pos), dev_i32(idx),
+    K.attn_fwd(d, qd, T, 0, kd, vd, NB, dev_i32(blk_len), dev_i32(blk_pos), dev_i32(idx),
                dev_i32(cnt), idx.shape[-1], w.mask, o, lse)
-    ws = torch.empty(K.attn_bwd_workspace(d, T, w.NB_phys, idx.shape[-1]), dtype=torch.uint8,
+    ws = torch.empty(K.attn_bwd_workspace(d, T, NB, idx.shape[-1]), dtype=torch.uint8,
                      device="cuda")
     dq = torch.empty(w.B, w.H, T, w.D, dtype=torch.float32, device="cuda")
-    dk = torch.empty(w.B, w.H, w.NB_phys, w.bs, w.D, dtype=torch.float32, device="cuda")
+    dk = torch.empty(w.B, w.H, NB, w.bs, w.D, dtype=torch.float32, device="cuda")
     dv = torch.empty_like(dk)
-    K.attn_bwd(d, qd, T, 0, kd, vd, w.NB_phys, dev_i32(blk_len), dev_i32(blk_pos), dev_i32(idx),
+    K.attn_bwd(d, qd, T, 0, kd, vd, NB, dev_i32(blk_len), dev_i32(blk_pos), dev_i32(idx),
                dev_i32(cnt), idx.shape[-1], w.mask, o, lse, dev_storage(dO, "bf16"), dq, dk, dv, ws)
     torch.cuda.synchronize()
     for (b, h) in [(0, 0), (1, 11)]:
         sl = (slice(b, b + 1), slice(h, h + 1))
         ro, rl = O.attention_fwd(q[sl], kpool[sl], vpool[sl], blk_len[sl], blk_pos[sl], idx[sl],
-                                 cnt[sl], w.scale, q_chunk=w.chunk_tokens)
+                                 cnt[sl], scale, q_chunk=w.chunk_tokens)
         mx, mean = _errs(host(o[sl]), ro)
         assert mx <= 2e-2 and mean <= 2e-3, ("o", mx, mean)
         rq, rk, rv = O.attention_bwd(q[sl], kpool[sl], vpool[sl], blk_len[sl], blk_pos[sl],
-                                     idx[sl], cnt[sl], dO[sl], w.scale, q_chunk=w.chunk_tokens)
+                                     idx[sl], cnt[sl], dO[sl], scale, q_chunk=w.chunk_tokens)
         for name, g, rf in (("dq", dq, rq), ("dk", dk, rk), ("dv", dv, rv)):
             ok, info = grad_ok(host(g[sl]), rf)
-            assert ok, (name, b, h, info)
-
-
-def _train_inputs(w):
-    chunks = [PI.chunk_tensors(w, t) for t in range(w.n_chunks)]
-    q = np.concatenate([c[0] for c in chunks], axis=2)
-    kpool = PI.pool_from_chunks(w, {t: c[1] for t, c in enumerate(chunks)})
-    vpool = PI.pool_from_chunks(w, {t: c[2] for t, c in enumerate(chunks)})
-    blk_len, blk_pos = PI.chunk_layout(w, range(w.n_chunks))
-    return q, kpool, vpool, blk_len, blk_pos
+            assert ok, (name, density, b, h, info)
 
 
 @pytest.mark.slow
 @pytest.mark.parametrize("density", [None, 0.10, 1.0])
 def test_train_lists_built_on_gpu_match_oracle(density):
     """The trainable path's lists, built by the library's own score/select calls
-    (one-shot per query chunk, or top fraction of allowed blocks), equal the
-    oracle's up to near-tie swaps."""
+    on a pool the engine filled through its own placement (one-shot per query
+    chunk, or top fraction of allowed blocks), equal the oracle's up to
+    near-tie swaps."""
     from block_sparse_attention_39_b200.engine import PbsaTrain
     w = PI.variant(PI.WORKLOADS["train"], B=1, H=4)
-    q, kpool, vpool, blk_len, blk_pos = _train_inputs(w)
+    q, kpool, vpool, blk_len, blk_pos, chunks = _train_inputs(w)
     T = PbsaTrain(w)
     T.q.copy_(dev_storage(q, "bf16"))
-    T.kpool.copy_(dev_storage(kpool, "bf16"))
-    T.vpool.copy_(dev_storage(vpool, "bf16"))
+    for t, c in enumerate(chunks):
+        T.write_chunk(t, dev_storage(c[1], "bf16"), dev_storage(c[2], "bf16"))
     T.set_meta()
     T.lists(density=density)
     torch.cuda.synchronize()
     idx, cnt = host(T.idx), host(T.cnt)
-    kb = O.pool_keys(kpool, blk_len, range(w.NB_phys), np.zeros((w.B, w.H, w.NB_phys, w.D)))
+    scale = 1 / math.sqrt(w.D)
+    NB = kpool.shape[2]
+    place = O.PoolPlacement(0, w.chunk_tokens, w.bs, w.W, w.n_chunks, ring=False)
+    nb_c = place.nb_c
+    kb = O.pool_keys(kpool, blk_len, range(NB), np.zeros((w.B, w.H, NB, w.D)))
     for t in range(w.n_chunks):
         qt = q[:, :, t * w.chunk_tokens:(t + 1) * w.chunk_tokens]
-        S = O.block_scores(O.pool_queries(qt, w.bs), kb, w.scale)
+        S = O.block_scores(O.pool_queries(qt, w.bs), kb, scale)
         m = O.memory_scores(S)
-        older = [p for c in range(0, max(0, t - w.W + 1)) for p in w.chunk_phys_ids(c)]
-        win = [p for c in w.window_chunks(t) for p in w.chunk_phys_ids(c)]
-        allowed = [p for c in range(t + 1) for p in w.chunk_phys_ids(c)]
+        older = [p for c in O.older_chunks(t, w.W) for p in place.chunk_ids(c)]
+        win = [p for c in O.window_chunks(t, w.W) for p in place.chunk_ids(c)]
+        allowed = [p for c in range(t + 1) for p in place.chunk_ids(c)]
         for h in range(w.H):
-            for i in range(w.nb_c):
-                r = t * w.nb_c + i
+            for i in range(nb_c):
+                r = t * nb_c + i
                 lst = [int(x) for x in idx[0, h, r, :cnt[0, h, r]]]
                 assert lst == sorted(set(lst))
                 if density is None:

@@ -32,53 +32,8 @@ def _status_clean():
     assert K.get_status() == 0
 
 
-class OracleRollout:
-    """The oracle's state of one layer's block pool, advanced chunk by chunk."""
-
-    def __init__(self, w):
-        self.w = w
-        NB = w.NB_phys
-        self.kp = np.zeros((w.B, w.H, NB, w.bs, w.D))
-        self.vp = np.zeros_like(self.kp)
-        self.bl = np.zeros((w.B, w.H, NB), dtype=np.int32)
-        self.bp = np.zeros((w.B, w.H, NB), dtype=np.int32)
-        self.kb = np.zeros((w.B, w.H, NB, w.D))
-        self.ss, self.sw = PI.empty_memory(w)
-        self.ss = self.ss.astype(np.int64)
-        self.sw = self.sw.astype(np.float64)
-
-    def write_chunk(self, t, k, v):
-        w = self.w
-        lens = w.chunk_block_lens()
-        for j, pid in enumerate(w.chunk_phys_ids(t)):
-            r0 = j * w.bs
-            self.kp[:, :, pid] = 0.0
-            self.vp[:, :, pid] = 0.0
-            self.kp[:, :, pid, :lens[j]] = k[:, :, r0:r0 + lens[j]]
-            self.vp[:, :, pid, :lens[j]] = v[:, :, r0:r0 + lens[j]]
-            self.bl[:, :, pid] = lens[j]
-            self.bp[:, :, pid] = t * w.chunk_tokens + j * w.bs
-
-    def step(self, t, q):
-        w = self.w
-        qb, self.kb, S, m = O.score_blocks(q, self.kp, self.bl, w.chunk_phys_ids(t), self.kb,
-                                           w.scale, w.bs)
-        c = w.leaving_chunk(t)
-        info = None
-        if c is not None:
-            out = O.update_memory(self.kp, self.vp, self.bl, self.bp, self.kb, self.ss, self.sw,
-                                  w.chunk_phys_ids(c), w.chunk_global_ids(c), m, w.P, w.n_sink,
-                                  w.policy, w.dtype)
-            self.kp, self.vp, self.bl, self.bp, self.kb, self.ss, self.sw, info = out
-        win = [p for cc in w.window_chunks(t) for p in w.chunk_phys_ids(cc)]
-        A = O.select_local(S, win, w.k, PI.mem_ids_all_slots(w), self.bl, w.mask,
-                           t * w.chunk_tokens, self.bp, w.bs, w.chunk_tokens)
-        idx, cnt = O.lists_to_arrays(A, PI.amax(w))
-        return dict(S=S, m=m, info=info, idx=idx, cnt=cnt)
-
-
-def _seed_gpu(L, orc):
-    w = orc.w
+def _seed_gpu(L, orc, w):
+    """The GPU layer's whole state set to the oracle's (the re-seeding)."""
     L.kpool.copy_(dev_storage(orc.kp, w.dtype))
     L.vpool.copy_(dev_storage(orc.vp, w.dtype))
     L.blk_len.copy_(dev_i32(orc.bl))
@@ -88,15 +43,19 @@ def _seed_gpu(L, orc):
     L.slot_w.copy_(torch.from_numpy(orc.sw.astype(np.float32)).cuda())
 
 
-def _compare_memory(L, orc, info, merged_tol):
-    w = orc.w
+def _compare_memory(L, orc, w, info, merged_tol):
     src, sw = host(L.slot_src), host(L.slot_w)
     kp, vp, bl, kb = host(L.kpool), host(L.vpool), host(L.blk_len), host(L.k_bar)
     exact = 0
     for b in range(w.B):
         for h in range(w.H):
             inf = info[(b, h)]
-            got = [int(x) for x in src[b, h] if x >= 0]
+            for s in range(w.n_sink):                   # sinks: pinned, never ranked
+                assert src[b, h, s] == orc.ss[b, h, s]
+                if orc.ss[b, h, s] >= 0:
+                    np.testing.assert_array_equal(kp[b, h, s], orc.kp[b, h, s])
+                    np.testing.assert_array_equal(vp[b, h, s], orc.vp[b, h, s])
+            got = [int(x) for x in src[b, h, w.n_sink:] if x >= 0]
             ok, same = band_ok(got, inf["keys"], len(inf["kept"]))
             assert ok, (b, h, sorted(got), sorted(inf["kept"]))
             assert len(got) <= w.P
@@ -122,32 +81,41 @@ def _compare_memory(L, orc, info, merged_tol):
     return exact
 
 
-def _run_rollout(w, steps, attn_steps):
-    orc = OracleRollout(w)
+def _run_rollout(w, steps, attn_steps, fused=False):
+    """Every step: the GPU state is re-seeded from the oracle's state after the
+    previous step, then each side writes chunk t through its own placement
+    (the engine's ``write_chunk``, the oracle's ``OracleLayer.write_chunk``)
+    and runs score -> update -> select (per call, or as one fused routing
+    call); the step's results are compared."""
+    orc = O.OracleLayer.of(w)
     L = PbsaLayer(w)
     merged_seen = 0
     for t in range(steps):
         q, k, v = PI.chunk_tensors(w, t)
+        _seed_gpu(L, orc, w)                    # state after step t-1
         orc.write_chunk(t, k, v)
-        _seed_gpu(L, orc)                       # state before this step, incl. the new chunk
+        L.write_chunk(t, dev_storage(k, w.dtype), dev_storage(v, w.dtype))
         L.q.copy_(dev_storage(q, w.dtype))
-        ref = orc.step(t, q)
-        L.score(t)
-        ci, cs = L.candidates(t)
-        L.update(ci, cs)
-        L.select(t)
+        ref = orc.step(t, q, attend=False)
+        if fused:
+            L.route(t)
+        else:
+            L.score(t)
+            ci, cs = L.candidates(t)
+            L.update(ci, cs)
+            L.select(t)
         torch.cuda.synchronize()
-        ids = w.chunk_phys_ids(t)
+        ids = orc.place.chunk_ids(t)
         np.testing.assert_allclose(host(L.scores)[:, :, :, ids], ref["S"][:, :, :, ids],
                                    rtol=1e-4, atol=1e-6)
         if ref["info"] is not None:
-            exact = _compare_memory(L, orc, ref["info"], merged_tol=2.0 ** -7)
+            exact = _compare_memory(L, orc, w, ref["info"], merged_tol=2.0 ** -7)
             assert exact >= w.B * w.H // 2, "too many near-tie differences"
             merged_seen += int((orc.sw > 1).sum())
         # local selection: band rule against the oracle's scores
         idx, cnt = host(L.idx), host(L.cnt)
         src = host(L.slot_src)
-        win = [p for c in w.window_chunks(t) for p in w.chunk_phys_ids(c)]
+        win = ref["win_ids"]
         for b in range(w.B):
             for h in range(w.H):
                 slots = [s for s in range(w.P) if src[b, h, s] >= 0]
@@ -160,16 +128,17 @@ def _run_rollout(w, steps, attn_steps):
                     assert ok, (t, b, h, i)
         if t in attn_steps:
             # attention on the oracle's post-update pool with the oracle's lists
-            dbf = K.dims(w.B, w.H, w.D, w.bs, w.scale, torch.bfloat16)
+            dbf = K.dims(w.B, w.H, w.D, w.bs, orc.scale, torch.bfloat16)
             o = torch.zeros(w.B, w.H, w.chunk_tokens, w.D, dtype=torch.bfloat16, device="cuda")
             lse = torch.zeros(w.B, w.H, w.chunk_tokens, dtype=torch.float32, device="cuda")
             K.attn_fwd(dbf, dev_storage(q, "bf16"), w.chunk_tokens, t * w.chunk_tokens,
-                       dev_storage(orc.kp, "bf16"), dev_storage(orc.vp, "bf16"), w.NB_phys,
+                       dev_storage(orc.kp, "bf16"), dev_storage(orc.vp, "bf16"), orc.place.NB,
                        dev_i32(orc.bl), dev_i32(orc.bp), dev_i32(ref["idx"]), dev_i32(ref["cnt"]),
                        ref["idx"].shape[-1], w.mask, o, lse)
             torch.cuda.synchronize()
-            ro, rl = O.attention_fwd(q, orc.kp, orc.vp, orc.bl, orc.bp, ref["idx"], ref["cnt"],
-                                     w.scale, w.mask, t * w.chunk_tokens)
+            ro, rl = O.attention_fwd(O.round_bf16(q), O.round_bf16(orc.kp), O.round_bf16(orc.vp),
+                                     orc.bl, orc.bp, ref["idx"], ref["cnt"], orc.scale, w.mask,
+                                     t * w.chunk_tokens)
             mx, mean = attn_errors(host(o), ro)
             assert mx <= ATT_MAX and mean <= ATT_MEAN, (t, mx, mean)
     return merged_seen
@@ -195,6 +164,7 @@ def test_free_running_rollout_invariants(fused):
     # structure and weights stay consistent at every step
     w = PI.WORKLOADS["rollout20s"]
     L = PbsaLayer(w)
+    nb_c = len(O.chunk_blocks(w.chunk_tokens, w.bs))
     admitted = 0
     for t in range(w.n_chunks):
         q, k, v = PI.chunk_tensors(w, t)
@@ -202,8 +172,8 @@ def test_free_running_rollout_invariants(fused):
         L.q.copy_(dev_storage(q, w.dtype))
         L.step(t, fused=fused)
         torch.cuda.synchronize()
-        if w.leaving_chunk(t) is not None:
-            admitted += w.nb_c
+        if O.leaving_chunk(t, w.W) is not None:
+            admitted += nb_c
         src, sw, bl = host(L.slot_src), host(L.slot_w), host(L.blk_len)
         cnt, idx = host(L.cnt), host(L.idx)
         for b in range(w.B):
@@ -213,6 +183,23 @@ def test_free_running_rollout_invariants(fused):
                 assert np.all(bl[b, h, :w.P][valid] > 0) and np.all(bl[b, h, :w.P][~valid] == 0)
                 # every admitted block is in exactly one slot's weight (merge policy)
                 assert abs(sw[b, h].sum() - admitted) < 1e-3
-                assert np.all(cnt[b, h] == valid.sum() + min(w.k, len(w.window_chunks(t)) * w.nb_c))
+                assert np.all(cnt[b, h] == valid.sum() + min(w.k, len(O.window_chunks(t, w.W)) * nb_c))
         o = host(L.o)
         assert np.isfinite(o).all()
+
+
+@pytest.mark.parametrize("policy", [PI.POLICY_EVICT, PI.POLICY_MERGE_MEAN])
+@pytest.mark.parametrize("fused", [False, True])
+def test_rollout_with_a_sink_slot(policy, fused):
+    # one pinned sink slot (block 0 of the rollout): block 0 leaves the window
+    # at step 2 and must land in slot 0 and stay there, never ranked out nor
+    # merged into, through both the per-call and the fused routing path
+    w = PI.variant(PI.WORKLOADS["tiny"], n_sink=1, policy=policy, rollout=True, n_chunks=7,
+                   seed=11)
+    _run_rollout(w, steps=7, attn_steps={2, 6}, fused=fused)
+
+
+def test_rollout_reseeded_with_token_mask_and_fp32():
+    # the tiny fp32 shape as a rollout under the token-causal mask
+    w = PI.variant(PI.WORKLOADS["tiny"], mask=PI.MASK_TOKEN, rollout=True, n_chunks=6, seed=12)
+    _run_rollout(w, steps=6, attn_steps={3, 5})

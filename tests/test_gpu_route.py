@@ -15,8 +15,8 @@ import torch
 import pbsa_inputs as PI
 from block_sparse_attention_39_b200 import pbsa as K
 from block_sparse_attention_39_b200.engine import PbsaLayer
-from tests.gpu_util import (ATT_MAX, ATT_MEAN, attn_errors, band_ok, dev_storage, host,
-                            load_layer, oracle_snapshot_step)
+from tests.gpu_util import (band_ok, check_step_attention, dev_storage, host, load_snapshot,
+                            oracle_snapshot_step)
 
 pytestmark = pytest.mark.gpu
 
@@ -45,17 +45,17 @@ def _barrier_words_zero(L):
 
 def _snapshot_pair(name):
     w = PI.WORKLOADS[name]
-    snap = PI.snapshot(w)
+    chunks = PI.snapshot_chunks(w)
     t = w.n_chunks - 1
     layers = []
     for _ in range(2):
         L = PbsaLayer(w)
-        load_layer(L, snap, w)
-        L.score(t, pool_ids=L.ids(("all",), snap["all_ids"]))   # cached pooled keys
+        load_snapshot(L, w, chunks)
+        L.score(t, pool_ids=L.all_ids())        # cached pooled keys
         L.reset_memory()
         layers.append(L)
     torch.cuda.synchronize()
-    return w, snap, t, layers
+    return w, chunks, t, layers
 
 
 def _per_call(L, t):
@@ -67,7 +67,7 @@ def _per_call(L, t):
 
 @pytest.mark.parametrize("name", ["tiny", "decode"])
 def test_route_equals_per_call_on_snapshot(name):
-    w, snap, t, (La, Lb) = _snapshot_pair(name)
+    w, chunks, t, (La, Lb) = _snapshot_pair(name)
     _per_call(La, t)
     Lb.route(t)
     torch.cuda.synchronize()
@@ -107,12 +107,12 @@ def test_route_equals_per_call_over_a_rollout(name, steps):
 
 
 def test_route_matches_oracle_on_decode_snapshot():
-    w, snap, t, (L, _) = _snapshot_pair("decode")
-    ref = oracle_snapshot_step(w, snap)
+    w, chunks, t, (L, _) = _snapshot_pair("decode")
+    ref = oracle_snapshot_step(w, chunks)
     L.route(t)
     L.attend(t)
     torch.cuda.synchronize()
-    ids = w.chunk_phys_ids(t)
+    ids = ref["new_ids"]
     np.testing.assert_allclose(host(L.scores)[..., ids], ref["S"][..., ids], rtol=1e-4, atol=1e-6)
     src = host(L.slot_src)
     for b in range(w.B):
@@ -120,13 +120,13 @@ def test_route_matches_oracle_on_decode_snapshot():
             inf = ref["info"][(b, h)]
             ok, _ = band_ok([int(x) for x in src[b, h] if x >= 0], inf["keys"], len(inf["kept"]))
             assert ok, (b, h)
-    if np.array_equal(host(L.idx), ref["idx"]) and np.array_equal(host(L.cnt), ref["cnt"]):
-        mx, mean = attn_errors(host(L.o), ref["O"])
-        assert mx <= ATT_MAX and mean <= ATT_MEAN, (mx, mean)
+    # attention checked unconditionally: against the oracle over the GPU's own
+    # lists and pool, and against the oracle's step when the lists agree
+    check_step_attention(L, w, ref, chunks[t][0])
 
 
 def test_route_inside_a_cuda_graph():
-    w, snap, t, (La, Lb) = _snapshot_pair("decode")
+    w, chunks, t, (La, Lb) = _snapshot_pair("decode")
     La.step(t, fused=False)
     s = torch.cuda.Stream()
     torch.cuda.synchronize()

@@ -486,3 +486,216 @@ def test_backward_all_kept_equals_torch_autograd(mask):
                 assert np.allclose(dv[b, h, j, :n], vt.grad[off:off + n].numpy(), atol=1e-11)
                 assert np.all(dk[b, h, j, n:] == 0)
                 off += n
+
+
+# --------------------------------------------------------------------------
+# block tiling of chunks (R9)
+# --------------------------------------------------------------------------
+
+def test_chunk_tiling_of_the_video_chunk():
+    # a chunk of 3 latent frames of 1560 tokens in 128-token blocks
+    blocks = O.chunk_blocks(4680, 128)
+    assert len(blocks) == 37
+    assert blocks[:2] == [(0, 128), (128, 128)]
+    assert blocks[-1] == (4608, 72)
+    assert all(n == 128 for _, n in blocks[:-1])
+    assert O.chunk_blocks(5, 64) == [(0, 5)]
+    assert O.chunk_blocks(128, 128) == [(0, 128)]
+    assert O.chunk_blocks(256, 64) == [(0, 64), (64, 64), (128, 64), (192, 64)]
+
+
+def test_query_blocks_tile_each_query_chunk_on_its_own():
+    # 500 query rows in chunks of 200 rows (the last chunk 100), blocks of 64:
+    # no block crosses a chunk boundary, each chunk ends in a short block
+    want = [(0, 64), (64, 64), (128, 64), (192, 8),
+            (200, 64), (264, 64), (328, 64), (392, 8),
+            (400, 64), (464, 36)]
+    assert O.query_blocks(500, 64, 200) == want
+    assert list(O.query_block_lengths(500, 64, 200)) == [n for _, n in want]
+    # one chunk (q_chunk 0) is the plain tiling
+    assert O.query_blocks(500, 64) == O.chunk_blocks(500, 64)
+    # the trainable shape: 7 chunks of 4680 tokens -> 7 x 37 = 259 blocks
+    tb = O.query_blocks(7 * 4680, 128, 4680)
+    assert len(tb) == 259
+    assert tb[36] == (4608, 72) and tb[37] == (4680, 128) and tb[-1] == (6 * 4680 + 4608, 72)
+
+
+def test_pooling_follows_the_query_chunk_tiling():
+    # rows of value r: each block's mean is the mean of its own row indices
+    q = np.arange(500, dtype=np.float64)[None, None, :, None] * np.ones((1, 1, 1, 3))
+    qb = O.pool_queries(q, 64, 200)
+    for i, (r0, n) in enumerate(O.query_blocks(500, 64, 200)):
+        assert np.allclose(qb[0, 0, i], r0 + (n - 1) / 2.0)
+    assert np.allclose(qb[0, 0, 3], 195.5)     # rows 192..199 only
+
+
+# --------------------------------------------------------------------------
+# the local window, the chunk leaving it, the pool placement (R7, R14)
+# --------------------------------------------------------------------------
+
+def test_window_and_leaving_chunk_by_hand_for_w2():
+    # W = 2: the current chunk and the one before it
+    table = {0: ([0], None, []), 1: ([0, 1], None, []), 2: ([1, 2], 0, [0]),
+             3: ([2, 3], 1, [0, 1]), 4: ([3, 4], 2, [0, 1, 2])}
+    for t, (win, gone, older) in table.items():
+        assert O.window_chunks(t, 2) == win
+        assert O.leaving_chunk(t, 2) == gone
+        assert O.older_chunks(t, 2) == older
+
+
+def test_window_other_sizes_and_every_chunk_leaves_once():
+    assert O.window_chunks(5, 1) == [5] and O.leaving_chunk(5, 1) == 4
+    assert O.window_chunks(1, 3) == [0, 1] and O.leaving_chunk(2, 3) is None
+    assert O.window_chunks(6, 3) == [4, 5, 6] and O.leaving_chunk(6, 3) == 3
+    for W in (1, 2, 3, 5):
+        left = [O.leaving_chunk(t, W) for t in range(40)]
+        left = [c for c in left if c is not None]
+        assert left == list(range(40 - W))      # each chunk leaves once, in order
+        for t in range(40):
+            assert len(O.window_chunks(t, W)) == min(W, t + 1)
+            assert sorted(O.older_chunks(t, W) + O.window_chunks(t, W)) == list(range(t + 1))
+
+
+def test_placement_by_hand_ring_and_snapshot():
+    ring = O.PoolPlacement(P=4, T_c=256, bs=64, W=2, n_chunks=9, ring=True)
+    assert ring.nb_c == 4 and ring.NB == 4 + 3 * 4
+    assert ring.chunk_ids(0) == [4, 5, 6, 7]
+    assert ring.chunk_ids(2) == [12, 13, 14, 15]
+    assert ring.chunk_ids(3) == [4, 5, 6, 7]
+    assert ring.global_ids(3) == [12, 13, 14, 15]
+    snap = O.PoolPlacement(P=24, T_c=4680, bs=128, W=2, n_chunks=5, ring=False)
+    assert snap.NB == 24 + 5 * 37 and snap.chunk_ids(4)[-1] == snap.NB - 1
+    assert snap.chunk_ids(1)[0] == 24 + 37
+
+
+def test_ring_keeps_the_leaving_chunk_readable():
+    # at every step the window chunks and the chunk leaving the window sit at
+    # pairwise different ring positions, so the update can still read it
+    for W in (1, 2, 4):
+        pl = O.PoolPlacement(P=3, T_c=100, bs=64, W=W, n_chunks=0, ring=True)
+        for t in range(30):
+            live = O.window_chunks(t, W) + [c for c in [O.leaving_chunk(t, W)] if c is not None]
+            firsts = [pl.chunk_ids(c)[0] for c in live]
+            assert len(set(firsts)) == len(live)
+            assert all(f >= pl.P for f in firsts)
+
+
+# --------------------------------------------------------------------------
+# packing of the attended lists
+# --------------------------------------------------------------------------
+
+def test_lists_to_arrays_pads_with_minus_one():
+    A = [[[[1, 5], [], [2]], [[0, 1, 2], [7], []]]]
+    idx, cnt = O.lists_to_arrays(A, 3)
+    assert idx.dtype == np.int32 and idx.shape == (1, 2, 3, 3)
+    assert idx[0, 0].tolist() == [[1, 5, -1], [-1, -1, -1], [2, -1, -1]]
+    assert idx[0, 1].tolist() == [[0, 1, 2], [7, -1, -1], [-1, -1, -1]]
+    assert cnt.tolist() == [[[2, 0, 1], [3, 1, 0]]]
+    with pytest.raises(ValueError):
+        O.lists_to_arrays([[[[1, 2, 3, 4]]]], 3)
+
+
+# --------------------------------------------------------------------------
+# the layer step (R14) and the trainable lists (R13, R18)
+# --------------------------------------------------------------------------
+
+def _tiny_layer(P=4, n_sink=0, policy=O.EVICT, W=2, k=2, ring=True, n_chunks=8):
+    return O.OracleLayer(1, 2, 8, 4, 10, P, n_sink, W, k, policy, O.MASK_CHUNK, "f64",
+                         n_chunks, ring)
+
+
+def test_rollout_step_admits_only_blocks_that_left_the_window():
+    r = np.random.default_rng(3)
+    L = _tiny_layer(P=3)
+    nb_c = L.place.nb_c                           # 10 tokens in blocks of 4: 3 blocks
+    assert nb_c == 3
+    for t in range(8):
+        q, k, v = (r.standard_normal((1, 2, 10, 8)) for _ in range(3))
+        L.write_chunk(t, k, v)
+        res = L.step(t, q)
+        gone = O.leaving_chunk(t, 2)
+        assert res["cand_src"] == ([] if gone is None else list(range(gone * 3, gone * 3 + 3)))
+        # every slot holds a block of a chunk that has left the window
+        left = {g for c in range(t + 1) if c not in O.window_chunks(t, 2) for g in range(3 * c, 3 * c + 3)}
+        for h in range(2):
+            held = [int(s) for s in L.ss[0, h] if s >= 0]
+            assert set(held) <= left
+            assert len(held) == min(3, len(left))
+            # the local part of each list is in the window; the rest are slots
+            for i in range(nb_c):
+                a = res["A"][0][h][i]
+                assert [x for x in a if x < 3] == [s for s in range(3) if L.ss[0, h, s] >= 0]
+                assert set(x for x in a if x >= 3) <= set(L.window_ids(t))
+                assert len([x for x in a if x >= 3]) == min(2, len(L.window_ids(t)))
+        # the row positions of the window blocks follow the chunk order
+        for c in O.window_chunks(t, 2):
+            ids = L.place.chunk_ids(c)
+            assert L.bp[0, 0, ids[0]] == 10 * c and L.bl[0, 0, ids[-1]] == 2
+
+
+def test_snapshot_step_offers_every_older_chunk():
+    r = np.random.default_rng(4)
+    L = _tiny_layer(P=4, ring=False, n_chunks=4)
+    for t in range(4):
+        _, k, v = (r.standard_normal((1, 2, 10, 8)) for _ in range(3))
+        L.write_chunk(t, k, v)
+    q = r.standard_normal((1, 2, 10, 8))
+    all_ids = [p for c in range(4) for p in L.place.chunk_ids(c)]
+    res = L.step(3, q, pool_ids=all_ids)
+    assert res["cand_src"] == list(range(6))      # chunks 0 and 1
+    assert res["cand_ids"] == L.place.chunk_ids(0) + L.place.chunk_ids(1)
+    assert res["win_ids"] == L.place.chunk_ids(2) + L.place.chunk_ids(3)
+
+
+def _train_case(seed, n_chunks=4, T_c=10, bs=4, H=2, D=8):
+    r = np.random.default_rng(seed)
+    q = r.standard_normal((1, H, n_chunks * T_c, D))
+    L = O.OracleLayer(1, H, D, bs, T_c, 0, 0, 2, 2, O.EVICT, O.MASK_CHUNK, "f64", n_chunks,
+                      ring=False)
+    for t in range(n_chunks):
+        L.write_chunk(t, r.standard_normal((1, H, T_c, D)), r.standard_normal((1, H, T_c, D)))
+    return q, L
+
+
+def test_trainable_lists_dense_and_budget_invariants():
+    q, L = _train_case(5)
+    nb_c, sc = L.place.nb_c, L.scale
+    # density 1: every chunk-causally allowed block
+    idx, cnt = O.trainable_lists(q, L.kp, L.bl, 10, 4, 2, 2, 2, sc, density=1.0)
+    for t in range(4):
+        allowed = list(range(0, (t + 1) * nb_c))
+        for i in range(nb_c):
+            r_ = t * nb_c + i
+            assert idx[0, 0, r_, :cnt[0, 0, r_]].tolist() == allowed
+    # budgets large enough: the one-shot lists are every allowed block too
+    idx, cnt = O.trainable_lists(q, L.kp, L.bl, 10, 4, 12, 2, 6, sc)
+    for t in range(4):
+        assert all(cnt[0, :, t * nb_c + i].tolist() == [(t + 1) * nb_c] * 2 for i in range(nb_c))
+    # small budgets: |A_i| = min(P, #older) + min(k, #window) and the persistent
+    # part is the exhaustive top-P of the chunk's memory score
+    P, k = 2, 2
+    idx, cnt = O.trainable_lists(q, L.kp, L.bl, 10, 4, P, 2, k, sc)
+    kb = O.pool_keys(L.kp, L.bl, range(L.place.NB), np.zeros((1, 2, L.place.NB, 8)))
+    for t in range(4):
+        older = [p for c in O.older_chunks(t, 2) for p in L.place.chunk_ids(c)]
+        win = [p for c in O.window_chunks(t, 2) for p in L.place.chunk_ids(c)]
+        S = O.block_scores(O.pool_queries(q[:, :, 10 * t:10 * t + 10], 4), kb, sc)
+        m = S.mean(axis=2)
+        for h in range(2):
+            top = sorted(older, key=lambda j: (-m[0, h, j], j))[:P]
+            for i in range(nb_c):
+                a = idx[0, h, t * nb_c + i, :cnt[0, h, t * nb_c + i]].tolist()
+                assert len(a) == min(P, len(older)) + min(k, len(win))
+                assert sorted(x for x in a if x in older) == sorted(top)
+                loc = sorted(win, key=lambda j: (-S[0, h, i, j], j))[:k]
+                assert sorted(x for x in a if x in win) == sorted(loc)
+
+
+def test_trainable_lists_density_counts():
+    q, L = _train_case(6)
+    nb_c = L.place.nb_c
+    for d in (0.05, 0.25, 0.5):
+        idx, cnt = O.trainable_lists(q, L.kp, L.bl, 10, 4, 2, 2, 2, L.scale, density=d)
+        for t in range(4):
+            n = (t + 1) * nb_c
+            assert np.all(cnt[0, :, t * nb_c:(t + 1) * nb_c] == math.ceil(d * n))

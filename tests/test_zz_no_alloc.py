@@ -6,9 +6,12 @@ never enter the CUDA allocator.  Its scratch is a fixed array of device memory
 inside the library, shared by every call.
 
 The GPU test calls it twice in a row through the C ABI, on two different
-problems, and checks each result against pbsa_attn_bwd (which takes a
-workspace from the caller) within the gradient tolerance of the backward
-tests; the second call would pick up the first call's leftovers if the shared
+problems.  Each result must equal, bit for bit, what pbsa_attn_bwd (which
+takes a workspace from the caller) gives on the same inputs -- both run the
+same kernels, which write dQ, dK and dV without atomics, so any difference
+would come from stale contents of the shared scratch -- and must match the
+CPU oracle's float64 gradients within the tolerance of the backward tests.
+The second call would pick up the first call's leftovers if the shared
 scratch were not cleared where it must start at zero.  This file is collected
 last so that a run stopping at its first failure has run every other test.
 """
@@ -53,13 +56,15 @@ def _problem(seed, B, H, D, bs, Tq, NB, Amax, mask):
     q_pos0 = int(bp[0, 0, -1])
     scale = 1 / math.sqrt(D)
     o, lse = O.attention_fwd(q, kp, vp, bl, bp, idx, cnt, scale, mask, q_pos0)
+    grads = O.attention_bwd(q, kp, vp, bl, bp, idx, cnt, dO, scale, mask, q_pos0)
     dev = lambda x: torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32)).cuda()
     i32 = lambda x: torch.from_numpy(np.ascontiguousarray(x, dtype=np.int32)).cuda()
     t = dict(q=dev(q).bfloat16(), kp=dev(kp).bfloat16(), vp=dev(vp).bfloat16(),
              o=dev(O.round_bf16(o)).bfloat16(), lse=dev(lse), dO=dev(dO).bfloat16(), bl=i32(bl),
              bp=i32(bp), idx=i32(idx), cnt=i32(cnt))
     d = K.dims(B, H, D, bs, scale, torch.bfloat16)
-    return d, t, dict(Tq=Tq, NB=NB, Amax=Amax, mask=mask, q_pos0=q_pos0, B=B, H=H, D=D, bs=bs)
+    return d, t, dict(Tq=Tq, NB=NB, Amax=Amax, mask=mask, q_pos0=q_pos0, B=B, H=H, D=D, bs=bs,
+                      oracle=grads)
 
 
 def _grads(meta):
@@ -110,9 +115,11 @@ def test_no_alloc_backward_matches_workspace_backward_twice():
              (2, 1, 3, 64, 64, 200, 7, 5, PI.MASK_CHUNK)]
     for seed, B, H, D, bs, Tq, NB, Amax, mask in cases:
         d, t, m = _problem(seed, B, H, D, bs, Tq, NB, Amax, mask)
-        ref = [x.cpu().numpy() for x in _with_workspace(d, t, m)]
-        got = [x.cpu().numpy() for x in _no_alloc(d, t, m)]
+        ref = _with_workspace(d, t, m)
+        got = _no_alloc(d, t, m)
         torch.cuda.synchronize()
-        for name, g, r in zip(("dq", "dk", "dv"), got, ref):
-            assert _close(g, r), (seed, name, float(np.abs(g - r).max()))
+        for name, g, r, o in zip(("dq", "dk", "dv"), got, ref, m["oracle"]):
+            assert torch.equal(g, r), (seed, name, float((g - r).abs().max()))
+            gh = g.double().cpu().numpy()
+            assert _close(gh, o), (seed, name, float(np.abs(gh - o).max()))
     assert K.get_status() == 0
