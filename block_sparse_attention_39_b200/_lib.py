@@ -66,6 +66,7 @@ SIGNATURES = {
                                       c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                                       c_void_p]),
     "pbsa_attn_bwd_noalloc_max_scratch": (c_size_t, []),
+    "pbsa_check_exp2": (c_int, [c_void_p, c_void_p, c_void_p, c_int, c_void_p]),
     "pbsa_get_status": (c_int, [c_void_p]),
     "pbsa_last_error": (ctypes.c_char_p, []),
     "pbsa_version": (ctypes.c_char_p, []),

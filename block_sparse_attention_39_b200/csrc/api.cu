@@ -8,6 +8,7 @@
 
 #include "common.cuh"
 #include "launch.h"
+#include "tc_sm100.cuh"
 #include "tmap.h"
 
 #include <cstdlib>
@@ -97,9 +98,36 @@ int make_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_
   return PBSA_OK;
 }
 
+// y_poly[i] = exp2_poly2(x[i]) (the FMA-pipe exponent of the attention
+// softmax), y_hw[i] = ex2.approx (the special-function unit it replaces on
+// three pairs in four), both on the device, for the unit test of the former.
+__global__ void exp2_check_kernel(const float* __restrict__ x, float* __restrict__ y_poly,
+                                  float* __restrict__ y_hw, int n) {
+  const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
+  if (i >= n) return;
+  const float x0 = x[i], x1 = (i + 1 < n) ? x[i + 1] : 0.f;
+  float p0, p1;
+  tc::f2_split(tc::exp2_poly2(tc::f2(x0, x1)), p0, p1);
+  y_poly[i] = p0;
+  y_hw[i] = tc::ex2(x0);
+  if (i + 1 < n) {
+    y_poly[i + 1] = p1;
+    y_hw[i + 1] = tc::ex2(x1);
+  }
+}
+
 }  // namespace pbsa
 
 extern "C" {
+
+int pbsa_check_exp2(const float* x, float* y_poly, float* y_hw, int n, void* stream) {
+  PBSA_CHECK_ARG(x && y_poly && y_hw && n >= 1, PBSA_ERR_ARG, "check_exp2: NULL buffer or n < 1");
+  const int pairs = (n + 1) / 2;
+  pbsa::exp2_check_kernel<<<(pairs + 255) / 256, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      x, y_poly, y_hw, n);
+  PBSA_CHECK_LAUNCH("exp2_check_kernel");
+  return PBSA_OK;
+}
 
 int pbsa_get_status(void* stream) {
   int* p = pbsa::device_status_ptr();

@@ -333,8 +333,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         // about 8k cycles each time it ran (measured with clock stamps).
         int lim = len;
         if (tok) lim = min(lim, max(0, qpos - kpos0 + 1));
+        if (__any_sync(0xffffffffu, lim < BS)) {
 #pragma unroll
-        for (int c = 0; c < BS; ++c) sr[c] = c < lim ? sr[c] : __float_as_uint(-INFINITY);
+          for (int c = 0; c < BS; ++c) sr[c] = c < lim ? sr[c] : __float_as_uint(-INFINITY);
+        }
       }
       float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll

@@ -47,22 +47,38 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// The same test, but a thread whose phase is not complete yet is suspended by
+// the hardware until the phase completes or about `hint_ns` pass, so a waiting
+// warp takes no issue slots from the warps that do the work.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity,
+                                                    uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
 // Bounded wait on an mbarrier phase.  Returns false (and raises the CTA's
 // abort flag and the device status word) when the time limit runs out, or
-// false at once when another thread of the CTA already aborted.
+// false at once when another thread of the CTA already aborted.  Each retry
+// sleeps in the hardware for up to 0.2 ms, so the abort flag and the clock
+// are read only a few times per wait.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
                                           int* status, int64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
-  uint64_t t0 = global_timer_ns();
-  for (uint32_t it = 0;; ++it) {
-    if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (;;) {
+    if (mbar_try_wait_sleep(bar, parity, 200000u)) return true;
     if (*abort_flag) return false;
-    if ((it & 63u) == 63u) {
-      if (static_cast<int64_t>(global_timer_ns() - t0) > limit_ns) {
-        *abort_flag = 1;
-        report_status(status, PBSA_ERR_TIMEOUT);
-        return false;
-      }
+    if (static_cast<int64_t>(global_timer_ns() - t0) > limit_ns) {
+      *abort_flag = 1;
+      report_status(status, PBSA_ERR_TIMEOUT);
+      return false;
     }
   }
 }
@@ -71,10 +87,11 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
 // MMAs already in flight).
 __device__ __forceinline__ bool mbar_drain(uint32_t bar, uint32_t parity, int* status,
                                            int64_t limit_ns) {
-  uint64_t t0 = global_timer_ns();
-  for (uint32_t it = 0;; ++it) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 63u) == 63u && static_cast<int64_t>(global_timer_ns() - t0) > limit_ns) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (;;) {
+    if (mbar_try_wait_sleep(bar, parity, 200000u)) return true;
+    if (static_cast<int64_t>(global_timer_ns() - t0) > limit_ns) {
       report_status(status, PBSA_ERR_TIMEOUT);
       return false;
     }
@@ -165,6 +182,16 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
       : "r"(taddr));
 }
 
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
+
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
@@ -244,6 +271,11 @@ __device__ __forceinline__ void mma_commit(uint32_t bar) {
       : "memory");
 }
 
+// Named barrier `id` (1..15) over `n` threads (a multiple of 32).
+__device__ __forceinline__ void named_bar(uint32_t id, uint32_t n) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+
 __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -287,18 +319,19 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
   return r;
 }
 
-// 2^x for a pair of x in [-126, 8], computed on the FMA pipe instead of the
+// 2^x for a pair of x in [-125, 8], computed on the FMA pipe instead of the
 // special-function unit.  Method: split x = n + f with n = round(x) by adding
 // and subtracting 1.5 * 2^23 (the sum's low mantissa bits hold n), evaluate a
 // degree-3 polynomial for 2^f on [-1/2, 1/2] (coefficients fitted for this
 // library by weighted least squares on Chebyshev nodes, max relative error
 // 7.6e-5, far below the 2^-9 of the bf16 P it feeds), and add n to the
-// exponent field.  Inputs below -126 are clamped (their value is below 2^-126).
+// exponent field.  Inputs below -125 are clamped to -125, so the result stays
+// a normal float (at most 2^-125, against a true value below that).
 __device__ __forceinline__ uint64_t exp2_poly2(uint64_t x) {
   float x0, x1;
   f2_split(x, x0, x1);
-  x0 = fmaxf(x0, -126.0f);
-  x1 = fmaxf(x1, -126.0f);
+  x0 = fmaxf(x0, -125.0f);
+  x1 = fmaxf(x1, -125.0f);
   const uint64_t xc = f2(x0, x1);
   const uint64_t magic = f2(12582912.0f, 12582912.0f);
   const uint64_t t = add2(xc, magic);                                  // round to integer

@@ -157,6 +157,12 @@ def attn_bwd_noalloc_max_scratch() -> int:
     return int(lib().pbsa_attn_bwd_noalloc_max_scratch())
 
 
+def check_exp2(x, y_poly, y_hw, stream=None):
+    """The softmax's FMA-pipe exponent and the special-function unit's, on x."""
+    _check("pbsa_check_exp2", lib().pbsa_check_exp2(_p(x), _p(y_poly), _p(y_hw), x.numel(),
+                                                     _s(stream)))
+
+
 def get_status(stream=None) -> int:
     """Synchronise the stream; return and clear the device status word."""
     return int(lib().pbsa_get_status(_s(stream)))

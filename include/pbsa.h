@@ -371,6 +371,15 @@ size_t pbsa_attn_bwd_noalloc_max_scratch(void);
  * clears it.  Returns PBSA_ERR_CUDA if the read itself fails. */
 int pbsa_get_status(void* stream);
 
+/* Checks the software exponent of the attention softmax.  For i < n:
+ * y_poly[i] = 2^x[i] as the softmax computes it on the FMA pipe for one pair of
+ * scores in four (a degree-3 polynomial after a Cody-Waite range split, stated
+ * relative error 7.6e-5 for x in [-125, 8]), y_hw[i] = 2^x[i] from the
+ * special-function unit (ex2.approx).  x, y_poly, y_hw: device float [n].
+ * Returns PBSA_ERR_ARG for NULL buffers or n < 1.  No counterpart on the
+ * pages: a test hook. */
+int pbsa_check_exp2(const float* x, float* y_poly, float* y_hw, int n, void* stream);
+
 /* Message for the last failing call made by this host thread ("" if none). */
 const char* pbsa_last_error(void);
 

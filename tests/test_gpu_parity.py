@@ -107,9 +107,22 @@ def test_update_memory_matches_oracle(key):
                 if src[b, h, s] < 0:
                     continue
                 assert bl[b, h, s] == ref["blk_len"][b, h, s]
-                np.testing.assert_array_equal(kp[b, h, s], ref["kpool"][b, h, s])
-                np.testing.assert_array_equal(vp[b, h, s], ref["vpool"][b, h, s])
-                np.testing.assert_allclose(kbar[b, h, s], ref["k_bar2"][b, h, s], rtol=1e-5, atol=1e-6)
+                if ref["slot_w"][b, h, s] == 1.0:
+                    # a copied block: exact
+                    np.testing.assert_array_equal(kp[b, h, s], ref["kpool"][b, h, s])
+                    np.testing.assert_array_equal(vp[b, h, s], ref["vpool"][b, h, s])
+                    np.testing.assert_allclose(kbar[b, h, s], ref["k_bar2"][b, h, s], rtol=1e-5,
+                                               atol=1e-6)
+                else:
+                    # a merged slot: the GPU averages in fp32, the oracle in fp64, both
+                    # round once to storage, so rows may differ by one storage ulp
+                    ulp = 2.0 ** -7 if w.dtype == "bf16" else 2.0 ** -22
+                    np.testing.assert_allclose(kp[b, h, s], ref["kpool"][b, h, s], rtol=ulp,
+                                               atol=1e-6)
+                    np.testing.assert_allclose(vp[b, h, s], ref["vpool"][b, h, s], rtol=ulp,
+                                               atol=1e-6)
+                    np.testing.assert_allclose(kbar[b, h, s], ref["k_bar2"][b, h, s], rtol=0,
+                                               atol=2e-3)
     assert exact >= (w.B * w.H + 1) // 2, "too many near-tie differences"
 
 

@@ -116,6 +116,7 @@ def _run_rollout(w, steps, attn_steps, fused=False):
         idx, cnt = host(L.idx), host(L.cnt)
         src = host(L.slot_src)
         win = ref["win_ids"]
+        qb = O.query_blocks(w.chunk_tokens, w.bs)
         for b in range(w.B):
             for h in range(w.H):
                 slots = [s for s in range(w.P) if src[b, h, s] >= 0]
@@ -123,8 +124,12 @@ def _run_rollout(w, steps, attn_steps, fused=False):
                     lst = [int(x) for x in idx[b, h, i, :cnt[b, h, i]]]
                     assert lst == sorted(set(lst))
                     assert [x for x in lst if x < w.P] == slots
-                    keys = {j: ref["S"][b, h, i, j] for j in win}
-                    ok, _ = band_ok([x for x in lst if x >= w.P], keys, min(w.k, len(win)))
+                    # token mask: only blocks that start at or before the block's last query
+                    last_q = t * w.chunk_tokens + qb[i][0] + qb[i][1] - 1
+                    cands = [j for j in win
+                             if w.mask == PI.MASK_CHUNK or orc.bp[b, h, j] <= last_q]
+                    keys = {j: ref["S"][b, h, i, j] for j in cands}
+                    ok, _ = band_ok([x for x in lst if x >= w.P], keys, min(w.k, len(cands)))
                     assert ok, (t, b, h, i)
         if t in attn_steps:
             # attention on the oracle's post-update pool with the oracle's lists
