@@ -208,11 +208,15 @@ class DecodeRunner:
         L.chunk_ids(self.t)
         torch.cuda.synchronize()
         self.flush_buf = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
-        # the per-call path (programmatic dependent launch between the kernels) is
-        # the faster schedule on this workload; the fused routing call is timed
-        # beside it in the breakdown
-        self.fused = False
-        self.launches_per_step = 6   # pool, score, plan, apply, select, attention
+        # the headline schedule: the routing call (one dependency-driven kernel for
+        # score -> update -> select) then attention; the per-call path (five
+        # kernels chained by programmatic dependent launch) is timed beside it
+        self.fused = True
+
+    @property
+    def launches_per_step(self):
+        # route_kernel + attention, or pool, score, plan, apply, select + attention
+        return 2 if self.fused else 6
 
     def step(self, ev=None, fused=None, appended=False):
         """One step.  fused: the routing call (pbsa_route_step) then attention;
@@ -756,32 +760,41 @@ def main():
     pk, pk_kind = peaks()
     runner = DecodeRunner(seed_offset=rank)
     w = runner.w
-    n_graphs = max(1, min(64, args.steps))
-    graphs, evs, s = runner.capture(n_graphs)
-    with torch.cuda.stream(s):
-        for i in range(args.warmup):
-            graphs[i % n_graphs].replay()
-    torch.cuda.synchronize()
-    clocks = ClockSampler(local)
-    barrier(world)
-    torch.cuda.synchronize()
-    clocks.start()
-    wall0 = time.perf_counter()
-    step_times = []
-    done = 0
-    while done < args.steps:
-        n = min(n_graphs, args.steps - done)
+
+    def timed_steps(fused, steps, clocks=None):
+        """Mean device time of `steps` whole steps (graphs with events only at the
+        step's start and end), after the warm-up."""
+        n_graphs = max(1, min(64, steps))
+        graphs, evs, s = runner.capture(n_graphs, fused=fused)
         with torch.cuda.stream(s):
-            for i in range(n):
-                graphs[i].replay()
+            for i in range(args.warmup):
+                graphs[i % n_graphs].replay()
         torch.cuda.synchronize()
-        step_times += [evs[i][0].elapsed_time(evs[i][-1]) for i in range(n)]
-        done += n
-    wall = time.perf_counter() - wall0
-    barrier(world)
-    clk = clocks.stop()
-    ms_step = float(np.mean(step_times))
-    del graphs
+        barrier(world)
+        torch.cuda.synchronize()
+        if clocks is not None:
+            clocks.start()
+        wall0 = time.perf_counter()
+        times = []
+        done = 0
+        while done < steps:
+            n = min(n_graphs, steps - done)
+            with torch.cuda.stream(s):
+                for i in range(n):
+                    graphs[i].replay()
+            torch.cuda.synchronize()
+            times += [evs[i][0].elapsed_time(evs[i][-1]) for i in range(n)]
+            done += n
+        wall = time.perf_counter() - wall0
+        barrier(world)
+        clk = clocks.stop() if clocks is not None else None
+        del graphs
+        return float(np.mean(times)), wall, clk
+
+    clocks = ClockSampler(local)
+    ms_step, wall, clk = timed_steps(runner.fused, args.steps, clocks)
+    # the other schedule, timed the same way on fewer steps (reported beside)
+    ms_other, _, _ = timed_steps(not runner.fused, min(args.steps, 200))
 
     def breakdown(fused):
         """Per-call times from separate graphs with events between the calls."""
@@ -829,6 +842,10 @@ def main():
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded N(0,1) Q/K/V, salience offsets N(0,2) on 10% of key blocks)",
         "config": config_of(w),
+        "ms_per_step_by_schedule": {
+            "routing kernel + attention": round(ms_step if runner.fused else ms_other, 5),
+            "per-call path + attention": round(ms_other if runner.fused else ms_step, 5),
+            "headline": "routing kernel + attention" if runner.fused else "per-call path + attention"},
         "per_call_ms": {"route_step": round(float(per[:, 0].mean()), 5),
                         "attn_fwd": round(ms_attn, 5),
                         "per_call_path": {

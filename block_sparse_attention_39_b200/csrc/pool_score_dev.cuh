@@ -260,12 +260,13 @@ __host__ __device__ inline int pool_stages(int bs) {
 }
 
 // Tiles of S: the per-call scoring kernel runs 32 x 32 tiles on 64-thread
-// CTAs (enough CTAs to cover the SMs on a decode step's few hundred tiles);
-// the fused routing kernel runs 64 x 64 tiles on its 256 threads.  Every
-// score and memory score is computed in the same order in both, so the two
-// give the same bits.
+// CTAs, 4 x 4 scores per thread (enough CTAs to cover the SMs on a decode
+// step's few hundred tiles); the fused routing kernel runs 32 x 32 tiles on its
+// 256 threads, 2 x 2 scores per thread, so a head's scores spread over more
+// SMs.  Every score and memory score is computed in the same order in both, so
+// the two give the same bits.
 constexpr int kScoreTile = 32, kScoreThreads = 64;
-constexpr int kRouteScoreTile = 64;
+constexpr int kRouteScoreTile = 32;
 
 struct ScoreArgs {
   const float* q_bar;
@@ -308,31 +309,51 @@ __device__ __forceinline__ void score_stage_wait() {
   asm volatile("cp.async.wait_group 0;\n" ::: "memory");
 }
 
+// <qm, k> of one key row, split over the four lanes of a quad (lane p takes
+// the float4 numbers p + 4m, one fmaf chain each) and combined as
+// (s0 + s1) + (s2 + s3).  All four lanes of the quad call it and get the sum.
+// Every memory score of the library is this function times the scale.
+template <int D>
+__device__ __forceinline__ float quad_dot(const float* qm, const float* k, int p) {
+  float s = 0.f;
+#pragma unroll
+  for (int m = 0; m < D / 16; ++m) {
+    const float4 x = *reinterpret_cast<const float4*>(qm + (p + 4 * m) * 4);
+    const float4 y = *reinterpret_cast<const float4*>(k + (p + 4 * m) * 4);
+    s = fmaf(x.x, y.x, s);
+    s = fmaf(x.y, y.y, s);
+    s = fmaf(x.z, y.z, s);
+    s = fmaf(x.w, y.w, s);
+  }
+  s += __shfl_xor_sync(0xffffffffu, s, 1);
+  s += __shfl_xor_sync(0xffffffffu, s, 2);
+  return s;
+}
+
 // One T x T tile of S: query blocks [T itile, +T) against key blocks
 // [T jblk, +T) of head bh, plus the memory scores of the query chunks that
-// start inside the tile's rows.  Called by all NT = T*T/16 threads of the CTA.
+// start inside the tile's rows.  Called by all NT = (T/R)^2 threads of the CTA.
 //
 // The tile is a small fp32 GEMM on the CUDA cores (K = D is short, and the
 // scores are compared against a selection threshold, so no reduced-precision
-// tensor-core inputs): thread (ty, tx) of the (T/4) x (T/4) grid owns rows
-// ty + (T/4) k and columns tx + (T/4) l (k, l < 4); every score is one fmaf
+// tensor-core inputs): thread (ty, tx) of the (T/R) x (T/R) grid owns rows
+// ty + (T/R) k and columns tx + (T/R) l (k, l < R); every score is one fmaf
 // chain over d = 0 .. D-1 in order, times scale.
 //
 // The memory score of chunk g is the mean of its scores over its query blocks.
 // The scores are linear in the pooled query, so that mean is computed as
 // scale * <mean of the chunk's pooled queries, k_bar_j> (equal up to rounding):
 // the chunk's mean query (sum in block order, fp32, then one divide), then one
-// dot per key block, split over four lanes (float4 number p + 4m to lane p)
-// and combined as (s0 + s1) + (s2 + s3).  The tile holding the chunk's first
-// query block does it, so no tile waits on another.
-template <int D, int T>
+// quad_dot per key block.  The tile holding the chunk's first query block does
+// it, so no tile waits on another.
+template <int D, int T, int R = 4>
 __device__ void score_item(const ScoreArgs& a, long bh, int jblk, int itile, float* ssm) {
   constexpr int PT = score_pitch<D>();
-  constexpr int G4 = T / 4, NT = G4 * G4;
+  constexpr int GR = T / R, NT = GR * GR;
   float* ks = ssm;                                         // [T][PT]
   float* qs = ks + T * PT;                                 // [T][PT]
   float* qm = qs + T * PT;                                 // [D] a chunk's mean query
-  const int t = threadIdx.x, tx = t % G4, ty = t / G4;
+  const int t = threadIdx.x, tx = t % GR, ty = t / GR;
   const int j0 = jblk * T, i0 = itile * T;
   const int nj = min(T, a.NB - j0), ni = min(T, a.nQB - i0);
   const float* qrows = a.q_bar + bh * a.nQB * D;
@@ -341,22 +362,22 @@ __device__ void score_item(const ScoreArgs& a, long bh, int jblk, int itile, flo
   score_stage<D, T, NT>(qs, qrows + static_cast<long>(i0) * D, ni);
   score_stage_wait();
   __syncthreads();
-  float acc[4][4];
+  float acc[R][R];
 #pragma unroll
-  for (int k = 0; k < 4; ++k)
+  for (int k = 0; k < R; ++k)
 #pragma unroll
-    for (int l = 0; l < 4; ++l) acc[k][l] = 0.f;
+    for (int l = 0; l < R; ++l) acc[k][l] = 0.f;
 #pragma unroll 4
   for (int d = 0; d < D; d += 4) {
-    float4 q[4], kk[4];
+    float4 q[R], kk[R];
 #pragma unroll
-    for (int k = 0; k < 4; ++k) q[k] = *reinterpret_cast<const float4*>(qs + (ty + G4 * k) * PT + d);
+    for (int k = 0; k < R; ++k) q[k] = *reinterpret_cast<const float4*>(qs + (ty + GR * k) * PT + d);
 #pragma unroll
-    for (int l = 0; l < 4; ++l) kk[l] = *reinterpret_cast<const float4*>(ks + (tx + G4 * l) * PT + d);
+    for (int l = 0; l < R; ++l) kk[l] = *reinterpret_cast<const float4*>(ks + (tx + GR * l) * PT + d);
 #pragma unroll
-    for (int k = 0; k < 4; ++k)
+    for (int k = 0; k < R; ++k)
 #pragma unroll
-      for (int l = 0; l < 4; ++l) {
+      for (int l = 0; l < R; ++l) {
         float s = acc[k][l];
         s = fmaf(q[k].x, kk[l].x, s);
         s = fmaf(q[k].y, kk[l].y, s);
@@ -366,11 +387,11 @@ __device__ void score_item(const ScoreArgs& a, long bh, int jblk, int itile, flo
       }
   }
 #pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    const int r = ty + G4 * k;
+  for (int k = 0; k < R; ++k) {
+    const int r = ty + GR * k;
 #pragma unroll
-    for (int l = 0; l < 4; ++l) {
-      const int c = tx + G4 * l;
+    for (int l = 0; l < R; ++l) {
+      const int c = tx + GR * l;
       if (r < ni && c < nj) a.scores[(bh * a.nQB + i0 + r) * a.NB + j0 + c] = acc[k][l] * a.scale;
     }
   }
@@ -405,18 +426,7 @@ __device__ void score_item(const ScoreArgs& a, long bh, int jblk, int itile, flo
     __syncthreads();
     const int p = t & 3;
     for (int c = t >> 2; c < T; c += NT / 4) {
-      float s = 0.f;
-#pragma unroll
-      for (int m = 0; m < D / 16; ++m) {
-        const float4 x = *reinterpret_cast<const float4*>(qm + (p + 4 * m) * 4);
-        const float4 y = *reinterpret_cast<const float4*>(ks + c * PT + (p + 4 * m) * 4);
-        s = fmaf(x.x, y.x, s);
-        s = fmaf(x.y, y.y, s);
-        s = fmaf(x.z, y.z, s);
-        s = fmaf(x.w, y.w, s);
-      }
-      s += __shfl_xor_sync(0xffffffffu, s, 1);
-      s += __shfl_xor_sync(0xffffffffu, s, 2);
+      const float s = quad_dot<D>(qm, ks + c * PT, p);
       if (p == 0 && c < nj) a.mem[(bh * a.groups + g) * a.NB + j0 + c] = s * a.scale;
     }
     __syncthreads();                  // qm free for the next chunk

@@ -71,6 +71,7 @@ extern "C" int pbsa_select_local(const pbsa_dims* d, const float* scores, int nQ
   a.nQB = nQB; a.NB = NB; a.n_win = n_win; a.k = k; a.n_mem = n_mem; a.mem_ld = mem_ld;
   a.mask = mask; a.q_pos0 = q_pos0; a.Tq = Tq; a.qc = d->q_chunk; a.bs = d->bs; a.Amax = Amax;
   a.qb_offset = qb_offset; a.nQB_total = nQB_total;
+  a.slot_len = nullptr; a.slot_pos = nullptr; a.slot_ld = 0; a.n_slot = 0;
 #define PBSA_SEL(WW, UU)                                                                       \
   if (W == WW && U == UU)                                                                      \
     err = launch(select_kernel<WW, UU>, grid, dim3(32 * kSelWarps), 0, st, a);

@@ -17,6 +17,12 @@
 
 #include "common.cuh"
 
+// Optional time stamps inside select_row for schedule studies (the fused
+// routing kernel defines this when built with -DPBSA_ROUTE_TRACE).
+#ifndef SEL_TRACE
+#define SEL_TRACE(i, bh, k) do {} while (0)
+#endif
+
 namespace pbsa {
 namespace dev {
 
@@ -34,18 +40,49 @@ struct SelArgs {
   int32_t* cnt;
   int* status;
   int nQB, NB, n_win, k, n_mem, mem_ld, mask, q_pos0, Tq, qc, bs, Amax, qb_offset, nQB_total;
+  // Optional (NULL in the per-call kernel): lengths and positions of ids
+  // 0..n_slot-1 taken from here (row bh at bh * slot_ld) instead of blk_len /
+  // blk_pos -- the fused routing kernel passes the values its memory update
+  // is writing, so the lists need not wait for the slot copies.
+  const int32_t* slot_len;
+  const int32_t* slot_pos;
+  long slot_ld;
+  int n_slot;
+};
+
+// Length (and position) of block id j of head bh as the selection reads them.
+__device__ __forceinline__ int sel_len(const SelArgs& a, long bh, int j) {
+  return (a.slot_len != nullptr && j < a.n_slot) ? a.slot_len[bh * a.slot_ld + j]
+                                                 : a.blk_len[bh * a.NB + j];
+}
+__device__ __forceinline__ int sel_pos(const SelArgs& a, long bh, int j) {
+  return (a.slot_len != nullptr && j < a.n_slot) ? a.slot_pos[bh * a.slot_ld + j]
+                                                 : a.blk_pos[bh * a.NB + j];
+}
+
+// No-op hook for select_row.
+struct NoWait {
+  __device__ bool operator()() const { return true; }
 };
 
 // The attended list of query block i of head bh, computed by one warp.
-template <int W, int U>
-__device__ __forceinline__ void select_row(const SelArgs& a, int i, long bh) {
-  const float* __restrict__ scores = a.scores;
-  const int32_t* __restrict__ win_ids = a.win_ids;
-  const int32_t* __restrict__ mem_ids = a.mem_ids;
-  const int32_t* __restrict__ blk_len = a.blk_len;
-  const int32_t* __restrict__ blk_pos = a.blk_pos;
-  int32_t* __restrict__ idx = a.idx;
-  int32_t* __restrict__ cnt = a.cnt;
+// `before_mem()` is called by every lane after the window's Top-K is sorted
+// and before any memory id's length is read; it returns false (warp-uniform)
+// to abandon the row.  The fused routing kernel waits there for the memory
+// update's plan, which states the slots' lengths; with slot lengths taken from
+// the plan, a window id below n_slot also waits, so its length is read after
+// the hook as well.
+template <int W, int U, typename Hook = NoWait>
+__device__ __forceinline__ void select_row(const SelArgs& a, int i, long bh,
+                                           Hook before_mem = Hook()) {
+  // plain pointers, no __restrict__: in the fused routing kernel the scores
+  // and block lengths are written earlier in the same launch, so they must not
+  // be read through the read-only data path
+  const float* scores = a.scores;
+  const int32_t* win_ids = a.win_ids;
+  const int32_t* mem_ids = a.mem_ids;
+  int32_t* idx = a.idx;
+  int32_t* cnt = a.cnt;
   int* status = a.status;
   const int NB = a.NB, n_win = a.n_win, k = a.k, n_mem = a.n_mem, mem_ld = a.mem_ld;
   const int mask = a.mask, q_pos0 = a.q_pos0, Tq = a.Tq, qc = a.qc, bs = a.bs;
@@ -72,38 +109,55 @@ __device__ __forceinline__ void select_row(const SelArgs& a, int i, long bh) {
     const int me = 32 * U - 1 - (lane * U + r);
     mid[r] = me < n_mem ? mem_ids[bh * mem_ld + me] : -1;
   }
-  int wlen[W], wpos[W], mlen[U];
-  float wsc[W];
+  // ---- Top-K over the window (element order is irrelevant before the sort)
+  uint64_t wkey[W];
+  int n_ok = 0;
+  auto window_topk = [&]() {
+    int wlen[W], wpos[W];
+    float wsc[W];
 #pragma unroll
-  for (int r = 0; r < W; ++r) {
-    const int j = wid[r];
-    const bool in = j >= 0 && j < NB;
-    if (r * 32 + lane < n_win && !in) report_status(status, PBSA_ERR_ARG);
-    wlen[r] = in ? blk_len[bh * NB + j] : 0;
-    wsc[r] = in ? srow[j] : 0.f;
-    wpos[r] = (in && mask == PBSA_MASK_TOKEN) ? blk_pos[bh * NB + j] : 0;
+    for (int r = 0; r < W; ++r) {
+      const int j = wid[r];
+      const bool in = j >= 0 && j < NB;
+      if (r * 32 + lane < n_win && !in) report_status(status, PBSA_ERR_ARG);
+      wlen[r] = in ? sel_len(a, bh, j) : 0;
+      wsc[r] = in ? srow[j] : 0.f;
+      wpos[r] = (in && mask == PBSA_MASK_TOKEN) ? sel_pos(a, bh, j) : 0;
+    }
+    n_ok = 0;
+#pragma unroll
+    for (int r = 0; r < W; ++r) {
+      bool ok = wlen[r] > 0;
+      if (mask == PBSA_MASK_TOKEN) ok = ok && wpos[r] <= last_q;
+      wkey[r] = ok ? score_key(wsc[r], static_cast<uint32_t>(wid[r])) : 0ull;
+      n_ok += ok ? 1 : 0;
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) n_ok += __shfl_xor_sync(0xffffffffu, n_ok, off);
+    warp_bitonic_sort_desc<W>(wkey);
+  };
+  bool win_late = false;
+  if (a.slot_len != nullptr) {
+    bool low = false;
+#pragma unroll
+    for (int r = 0; r < W; ++r) low = low || (wid[r] >= 0 && wid[r] < a.n_slot);
+    win_late = __any_sync(0xffffffffu, low);
   }
+  SEL_TRACE(i, bh, 0);
+  if (!win_late) window_topk();
+  SEL_TRACE(i, bh, 1);
+  if (!before_mem()) return;
+  SEL_TRACE(i, bh, 2);
+  if (win_late) window_topk();
+  const int take = min(k, n_ok);
+  int mlen[U];
 #pragma unroll
   for (int r = 0; r < U; ++r) {
     const int m = mid[r];
     // -1 names no block; any other id outside the pool is an argument error
     if (m >= NB || m < -1) report_status(status, PBSA_ERR_ARG);
-    mlen[r] = (m >= 0 && m < NB) ? blk_len[bh * NB + m] : 0;
+    mlen[r] = (m >= 0 && m < NB) ? sel_len(a, bh, m) : 0;
   }
-  // ---- Top-K over the window (element order is irrelevant before the sort)
-  uint64_t wkey[W];
-  int n_ok = 0;
-#pragma unroll
-  for (int r = 0; r < W; ++r) {
-    bool ok = wlen[r] > 0;
-    if (mask == PBSA_MASK_TOKEN) ok = ok && wpos[r] <= last_q;
-    wkey[r] = ok ? score_key(wsc[r], static_cast<uint32_t>(wid[r])) : 0ull;
-    n_ok += ok ? 1 : 0;
-  }
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) n_ok += __shfl_xor_sync(0xffffffffu, n_ok, off);
-  warp_bitonic_sort_desc<W>(wkey);
-  const int take = min(k, n_ok);
 
   // ---- union with the memory ids, ascending (descending sort of ~id).
   // Sorted window element e (lane e / W, register e % W) moves to union
@@ -127,7 +181,9 @@ __device__ __forceinline__ void select_row(const SelArgs& a, int i, long bh) {
     }
     key[r] = nk;
   }
+  SEL_TRACE(i, bh, 3);
   warp_bitonic_sort_desc<U>(key);
+  SEL_TRACE(i, bh, 4);
 
   // ---- dedupe and write
   uint64_t prev_last = __shfl_up_sync(0xffffffffu, key[U - 1], 1);
@@ -163,6 +219,148 @@ __device__ __forceinline__ void select_row(const SelArgs& a, int i, long bh) {
   }
   for (int e = total + lane; e < Amax; e += 32) out[e] = -1;
   if (lane == 0) cnt[bh * nQB_total + qb_offset + i] = total;
+  SEL_TRACE(i, bh, 5);
+}
+
+// Shared memory per warp of select_row_bitmap: 32*W window keys and a bitmap
+// of kSelBmWords words (block ids below 32 * kSelBmWords).
+constexpr int kSelBmWords = 1024;
+template <int W>
+__host__ __device__ constexpr int sel_bitmap_smem_per_warp() {
+  return 32 * W * 8 + kSelBmWords * 4;
+}
+
+// The same list as select_row, computed without sorting: the window's Top-K
+// by counting, for each candidate, the keys larger than its own (keys are
+// unique: the id is in the low bits), and the union with the memory ids as a
+// bitmap over block ids, emitted in ascending order with a popcount prefix
+// scan (duplicates merge in the bitmap).  Needs NB <= 32 * kSelBmWords.
+// `wsm` is this warp's shared memory (sel_bitmap_smem_per_warp<W>() bytes).
+template <int W, int U, typename Hook = NoWait>
+__device__ __forceinline__ void select_row_bitmap(const SelArgs& a, int i, long bh, uint8_t* wsm,
+                                                  Hook before_mem = Hook()) {
+  uint64_t* skeys = reinterpret_cast<uint64_t*>(wsm);                 // [32*W]
+  uint32_t* bm = reinterpret_cast<uint32_t*>(wsm + 32 * W * 8);       // [kSelBmWords]
+  const int NB = a.NB, n_win = a.n_win, n_mem = a.n_mem;
+  const int lane = threadIdx.x & 31;
+  const float* srow = a.scores + (bh * a.nQB_total + a.qb_offset + i) * static_cast<long>(NB);
+  int qrow0, qlen;
+  qb_rows(i, a.Tq, a.qc, a.bs, qrow0, qlen);
+  const int last_q = a.q_pos0 + qrow0 + qlen - 1;
+  const int nbw = (NB + 31) / 32;
+
+  int wid[W], mid[U];
+#pragma unroll
+  for (int r = 0; r < W; ++r) {
+    const int e = lane + 32 * r;
+    wid[r] = e < n_win ? a.win_ids[e] : -1;
+  }
+#pragma unroll
+  for (int r = 0; r < U; ++r) {
+    const int me = lane + 32 * r;
+    mid[r] = me < n_mem ? a.mem_ids[bh * a.mem_ld + me] : -1;
+  }
+  // the bitmap starts empty
+  for (int w = lane; w < nbw; w += 32) bm[w] = 0u;
+  uint64_t wkey[W];
+  bool wsel[W];
+  auto window_topk = [&]() {
+    int n_ok = 0;
+#pragma unroll
+    for (int r = 0; r < W; ++r) {
+      const int j = wid[r];
+      const bool in = j >= 0 && j < NB;
+      if (r * 32 + lane < n_win && !in) report_status(a.status, PBSA_ERR_ARG);
+      const int len = in ? sel_len(a, bh, j) : 0;
+      const float sc = in ? srow[j] : 0.f;
+      const int pos = (in && a.mask == PBSA_MASK_TOKEN) ? sel_pos(a, bh, j) : 0;
+      bool ok = len > 0;
+      if (a.mask == PBSA_MASK_TOKEN) ok = ok && pos <= last_q;
+      wkey[r] = ok ? score_key(sc, static_cast<uint32_t>(j)) : 0ull;
+      skeys[lane + 32 * r] = wkey[r];
+      n_ok += __popc(__ballot_sync(0xffffffffu, ok));
+    }
+    __syncwarp();
+    const int take = min(a.k, n_ok);
+    // rank = number of larger keys; two keys per 16-byte shared load
+    int rank[W];
+#pragma unroll
+    for (int r = 0; r < W; ++r) rank[r] = 0;
+    const ulonglong2* k2 = reinterpret_cast<const ulonglong2*>(skeys);
+#pragma unroll 4
+    for (int f = 0; f < 16 * W; ++f) {
+      const ulonglong2 v = k2[f];
+#pragma unroll
+      for (int r = 0; r < W; ++r) rank[r] += (v.x > wkey[r] ? 1 : 0) + (v.y > wkey[r] ? 1 : 0);
+    }
+#pragma unroll
+    for (int r = 0; r < W; ++r) wsel[r] = wkey[r] != 0ull && rank[r] < take;
+  };
+  bool win_late = false;
+  if (a.slot_len != nullptr) {
+    bool low = false;
+#pragma unroll
+    for (int r = 0; r < W; ++r) low = low || (wid[r] >= 0 && wid[r] < a.n_slot);
+    win_late = __any_sync(0xffffffffu, low);
+  }
+  SEL_TRACE(i, bh, 0);
+  if (!win_late) window_topk();
+  SEL_TRACE(i, bh, 1);
+  if (!before_mem()) return;
+  SEL_TRACE(i, bh, 2);
+  if (win_late) window_topk();
+  __syncwarp();                               // the bitmap is zero
+#pragma unroll
+  for (int r = 0; r < W; ++r)
+    if (wsel[r]) atomicOr(&bm[wid[r] >> 5], 1u << (wid[r] & 31));
+#pragma unroll
+  for (int r = 0; r < U; ++r) {
+    const int m = mid[r];
+    // -1 names no block; any other id outside the pool is an argument error
+    if (m >= NB || m < -1) report_status(a.status, PBSA_ERR_ARG);
+    if (m >= 0 && m < NB && sel_len(a, bh, m) > 0) atomicOr(&bm[m >> 5], 1u << (m & 31));
+  }
+  __syncwarp();
+  SEL_TRACE(i, bh, 3);
+  // ---- count, then write the ids in ascending order
+  int total = 0;
+  for (int w0 = 0; w0 < nbw; w0 += 32) {
+    const uint32_t word = w0 + lane < nbw ? bm[w0 + lane] : 0u;
+    int c = __popc(word);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) c += __shfl_xor_sync(0xffffffffu, c, off);
+    total += c;
+  }
+  int32_t* out = a.idx + (bh * a.nQB_total + a.qb_offset + i) * static_cast<long>(a.Amax);
+  int32_t* cnt = a.cnt + bh * a.nQB_total + a.qb_offset + i;
+  if (total > a.Amax) {
+    if (lane == 0) report_status(a.status, PBSA_ERR_SHAPE);
+    for (int e = lane; e < a.Amax; e += 32) out[e] = -1;
+    if (lane == 0) *cnt = 0;
+    return;
+  }
+  int base = 0;
+  for (int w0 = 0; w0 < nbw; w0 += 32) {
+    uint32_t word = w0 + lane < nbw ? bm[w0 + lane] : 0u;
+    const int c = __popc(word);
+    int incl = c;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += v;
+    }
+    int pos = base + incl - c;
+    while (word) {
+      const int b = __ffs(word) - 1;
+      out[pos++] = (w0 + lane) * 32 + b;
+      word &= word - 1u;
+    }
+    base += __shfl_sync(0xffffffffu, incl, 31);
+  }
+  for (int e = total + lane; e < a.Amax; e += 32) out[e] = -1;
+  if (lane == 0) *cnt = total;
+  SEL_TRACE(i, bh, 4);
+  SEL_TRACE(i, bh, 5);
 }
 
 }  // namespace dev

@@ -25,6 +25,12 @@
 
 #include "common.cuh"
 
+// Optional time stamps inside plan_head for schedule studies (the fused
+// routing kernel defines this when built with -DPBSA_ROUTE_TRACE).
+#ifndef PLAN_TRACE
+#define PLAN_TRACE(bh, k) do {} while (0)
+#endif
+
 namespace pbsa {
 namespace dev {
 
@@ -41,17 +47,19 @@ struct PlanView {
   int32_t* moff;      // [P + 1] merge list offsets
   int32_t* mref;      // [M] physical id, or -(1 + s) for stash entry s
   int32_t* mlen;      // [M]
+  int32_t* nlen;      // [P] the slot's blk_len after the update
+  int32_t* npos;      // [P] the slot's blk_pos after the update
   float* base_w;      // [P]
   float* mw;          // [M]
 };
 
 __host__ __device__ inline size_t plan_bytes(int P, int M) {
-  size_t ints = 7 * static_cast<size_t>(P) + 1 + 2 * static_cast<size_t>(M);
+  size_t ints = 9 * static_cast<size_t>(P) + 1 + 2 * static_cast<size_t>(M);
   size_t flts = static_cast<size_t>(P) + static_cast<size_t>(M);
   return ((ints + flts) * 4 + 255) / 256 * 256;
 }
 
-__device__ inline PlanView plan_view(void* ws, long bh, int P, int M) {
+__host__ __device__ inline PlanView plan_view(void* ws, long bh, int P, int M) {
   char* p = static_cast<char*>(ws) + bh * plan_bytes(P, M);
   int32_t* ip = reinterpret_cast<int32_t*>(p);
   PlanView v;
@@ -64,6 +72,8 @@ __device__ inline PlanView plan_view(void* ws, long bh, int P, int M) {
   v.moff = ip; ip += P + 1;
   v.mref = ip; ip += M;
   v.mlen = ip; ip += M;
+  v.nlen = ip; ip += P;
+  v.npos = ip; ip += P;
   float* fp = reinterpret_cast<float*>(ip);
   v.base_w = fp; fp += P;
   v.mw = fp;
@@ -117,7 +127,7 @@ __host__ __device__ inline size_t merge_key_smem(int P, int D) {
 }
 
 // Shared memory of plan_head (one (b,h) at a time, 256 threads).
-struct PlanSmem {
+struct __align__(16) PlanSmem {
   uint64_t skey[kMaxItems];
   int it_phys[kMaxItems], it_src[kMaxItems], it_old[kMaxItems], it_len[kMaxItems];
   int it_pos[kMaxItems];
@@ -129,6 +139,7 @@ struct PlanSmem {
   int free_pos[256];
   int sink_item[256];
   int tcount[256];
+  int tmaxlen[256];            // longest loser merged into slot s
   int s_op[256];
   int s_moff[256];
   int s_tot[8];
@@ -136,8 +147,12 @@ struct PlanSmem {
 };
 
 // The update plan of head bh, written to its part of the workspace.  `sk`
-// holds P*D floats (kept pooled keys, merge policy only).
-__device__ inline void plan_head(const UpdArgs& a, long bh, PlanSmem& sm, float* sk) {
+// holds P*D floats (kept pooled keys, merge policy only).  `item_mem`, if not
+// NULL, holds the memory score of every plan item (occupied non-sink slots,
+// then the candidates), computed by the caller; otherwise they are read from
+// a.mem.
+__device__ inline void plan_head(const UpdArgs& a, long bh, PlanSmem& sm, float* sk,
+                                 const float* item_mem = nullptr) {
   uint64_t* skey = sm.skey;
   int* it_phys = sm.it_phys;
   int* it_src = sm.it_src;
@@ -152,11 +167,13 @@ __device__ inline void plan_head(const UpdArgs& a, long bh, PlanSmem& sm, float*
   int* free_pos = sm.free_pos;
   int* sink_item = sm.sink_item;
   int* tcount = sm.tcount;
+  int* tmaxlen = sm.tmaxlen;
   int* s_op = sm.s_op;
   int* s_moff = sm.s_moff;
   int* s_tot = sm.s_tot;
   int& s_nvalid = sm.s_nvalid;
   __syncthreads();   // shared memory may still be read by the previous item
+  PLAN_TRACE(bh, 0);
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
   const int P = a.P, n_sink = a.n_sink;
   const int n_dyn = P - n_sink;
@@ -201,7 +218,7 @@ __device__ inline void plan_head(const UpdArgs& a, long bh, PlanSmem& sm, float*
     }
     it_pos[t] = pos;
     if (valid) {
-      const float m = a.mem[bh * a.NB + phys];
+      const float m = item_mem ? item_mem[t] : a.mem[bh * a.NB + phys];
       key = (static_cast<uint64_t>(orderable(m)) << 32) |
             (static_cast<uint64_t>(0xffffffu - static_cast<uint32_t>(src)) << 8) |
             static_cast<uint64_t>(t);
@@ -212,12 +229,21 @@ __device__ inline void plan_head(const UpdArgs& a, long bh, PlanSmem& sm, float*
   __syncthreads();
 
   // ---- rank: keys are unique (item index in the low bits), so an item's
+  PLAN_TRACE(bh, 1);
   // position in the descending order is the number of larger keys; all 256
   // threads count at once.
   {
     const uint64_t mine = skey[t];
     int rank = 0;
-    for (int u = 0; u < NI; ++u) rank += skey[u] > mine ? 1 : 0;
+    // keys past NI are zero and never larger; 8 keys per step, all loads first
+    const ulonglong2* k2 = reinterpret_cast<const ulonglong2*>(skey);
+    for (int u2 = 0; u2 < (NI + 7) / 8 * 4; u2 += 4) {
+      ulonglong2 v[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) v[q] = k2[u2 + q];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) rank += (v[q].x > mine ? 1 : 0) + (v[q].y > mine ? 1 : 0);
+    }
     if (mine != 0) it_rank[t] = rank;
     const int nv = __syncthreads_count(mine != 0 ? 1 : 0);
     if (t == 0) s_nvalid = nv;
@@ -227,6 +253,7 @@ __device__ inline void plan_head(const UpdArgs& a, long bh, PlanSmem& sm, float*
   const int n_keep = min(n_dyn, n_valid);
 
   // ---- kept old slots stay; list the free non-sink slots in ascending order
+  PLAN_TRACE(bh, 2);
   if (t < NI && it_rank[t] >= 0 && it_rank[t] < n_keep && it_old[t] >= 0) {
     it_slot[t] = it_old[t];
     holder[it_old[t]] = t;
@@ -264,6 +291,7 @@ __device__ inline void plan_head(const UpdArgs& a, long bh, PlanSmem& sm, float*
   __syncthreads();
 
   // ---- merge targets: most similar kept slot by pooled-key dot product
+  PLAN_TRACE(bh, 3);
   // (ties -> lowest slot).  The kept blocks' pooled keys are staged in shared
   // memory with a padded row stride; each warp takes one loser at a time, its
   // lanes take one slot each (a full dot product over D, in dimension order),
@@ -339,18 +367,24 @@ __device__ inline void plan_head(const UpdArgs& a, long bh, PlanSmem& sm, float*
   if (merging && t < NI && it_rank[t] >= n_keep) rank_item[it_rank[t] - n_keep] = t;
   __syncthreads();
   for (int s = warp; s < P; s += 8) {
-    int n = 0;
+    int n = 0, mx = 0;
     if (merging) {
       for (int c0 = 0; c0 < n_lose; c0 += 32) {
         const int u = c0 + lane < n_lose ? rank_item[c0 + lane] : -1;
-        n += __popc(__ballot_sync(0xffffffffu, u >= 0 && it_target[u] == s));
+        const bool hit = u >= 0 && it_target[u] == s;
+        n += __popc(__ballot_sync(0xffffffffu, hit));
+        mx = max(mx, __reduce_max_sync(0xffffffffu, hit ? it_len[u] : 0));
       }
     }
-    if (lane == 0) tcount[s] = n;
+    if (lane == 0) {
+      tcount[s] = n;
+      tmaxlen[s] = mx;
+    }
   }
   __syncthreads();
 
   // ---- per-slot plan (thread s plans slot s)
+  PLAN_TRACE(bh, 4);
   if (t < P) {
     const int s = t;
     int op = OP_NONE, base = -1, blen = 0, src = -1, pos = 0;
@@ -374,6 +408,17 @@ __device__ inline void plan_head(const UpdArgs& a, long bh, PlanSmem& sm, float*
     s_op[s] = op;
     pv.op[s] = op; pv.base[s] = base; pv.base_len[s] = blen; pv.base_w[s] = bw;
     pv.src[s] = src; pv.pos[s] = pos; pv.stash[s] = 0;
+    // what apply_item will leave in blk_len / blk_pos of the slot
+    int nl = 0, np = 0;
+    if (op == OP_NONE) {
+      nl = a.blk_len[bh * a.NB + s];
+      np = a.blk_pos[bh * a.NB + s];
+    } else if (op == OP_WRITE) {
+      nl = tcount[s] > 0 ? max(blen, tmaxlen[s]) : blen;
+      np = pos;
+    }
+    pv.nlen[s] = nl;
+    pv.npos[s] = np;
   }
   const int v = (t < P) ? tcount[t] : 0;
   int total = 0;
@@ -410,7 +455,9 @@ __device__ inline void plan_head(const UpdArgs& a, long bh, PlanSmem& sm, float*
 
 // -------------------------------------------------------------------- stash
 // Copy slot s of head bh to the stash when the plan asks for it.
-template <typename T>
+// CB: 16-byte chunks of K and of V each thread holds per round (the fused
+// routing kernel runs with fewer registers and passes a smaller batch).
+template <typename T, int CB = 8>
 __device__ void stash_item(const UpdArgs& a, int s, long bh, const T* __restrict__ kpool,
                            const T* __restrict__ vpool, T* __restrict__ stash) {
   PlanView pv = plan_view(a.ws, bh, a.P, a.M);
@@ -420,15 +467,15 @@ __device__ void stash_item(const UpdArgs& a, int s, long bh, const T* __restrict
   const uint4* vs = reinterpret_cast<const uint4*>(vpool + (bh * a.NB + s) * static_cast<long>(a.bs) * a.D);
   uint4* kd = reinterpret_cast<uint4*>(stash + ((bh * a.P + s) * 2 + 0) * static_cast<long>(a.bs) * a.D);
   uint4* vd = reinterpret_cast<uint4*>(stash + ((bh * a.P + s) * 2 + 1) * static_cast<long>(a.bs) * a.D);
-  for (int e0 = 0; e0 < n16; e0 += 256 * 8) {
-    uint4 ka[8], va[8];
+  for (int e0 = 0; e0 < n16; e0 += 256 * CB) {
+    uint4 ka[CB], va[CB];
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
+    for (int k = 0; k < CB; ++k) {
       const int e = e0 + threadIdx.x + k * 256;
       if (e < n16) { ka[k] = ks[e]; va[k] = vs[e]; }
     }
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
+    for (int k = 0; k < CB; ++k) {
       const int e = e0 + threadIdx.x + k * 256;
       if (e < n16) { kd[e] = ka[k]; vd[e] = va[k]; }
     }
@@ -481,11 +528,12 @@ struct Elem<float> {
 };
 
 // Write slot s of head bh as planned (copy, weighted mean or clear) and update
-// its pooled key and metadata.  `red` holds 8*D floats; s_mref, s_mlen and
+// its pooled key and metadata.  A plain copy moves CB 16-byte chunks of K and
+// of V per thread per round.  `red` holds 8*D floats; s_mref, s_mlen and
 // s_mw are shared arrays of kMaxItems entries for the slot's merge list.
-template <typename T, int D>
+template <typename T, int D, int CB = 8>
 __device__ void apply_item(const UpdArgs& a, int s, long bh, T* __restrict__ kpool,
-                           T* __restrict__ vpool, const T* __restrict__ stash,
+                           T* __restrict__ vpool, const T* stash,
                            int32_t* __restrict__ blk_len, int32_t* __restrict__ blk_pos,
                            float* __restrict__ k_bar, int32_t* __restrict__ slot_src,
                            float* __restrict__ slot_w, float (*red)[D], int* s_mref,
@@ -525,10 +573,10 @@ __device__ void apply_item(const UpdArgs& a, int s, long bh, T* __restrict__ kpo
     // source and destination are different blocks of the same pool: load a
     // batch of 16-byte chunks into registers, then store them
     const int n16 = static_cast<int>(blk_elems * sizeof(T) / 16);
-    for (int e0 = 0; e0 < n16; e0 += 256 * 8) {
-      uint4 ka[8], va[8];
+    for (int e0 = 0; e0 < n16; e0 += 256 * CB) {
+      uint4 ka[CB], va[CB];
 #pragma unroll
-      for (int k = 0; k < 8; ++k) {
+      for (int k = 0; k < CB; ++k) {
         const int e = e0 + t + k * 256;
         if (e < n16) {
           ka[k] = reinterpret_cast<const uint4*>(kb)[e];
@@ -536,7 +584,7 @@ __device__ void apply_item(const UpdArgs& a, int s, long bh, T* __restrict__ kpo
         }
       }
 #pragma unroll
-      for (int k = 0; k < 8; ++k) {
+      for (int k = 0; k < CB; ++k) {
         const int e = e0 + t + k * 256;
         if (e < n16) {
           reinterpret_cast<uint4*>(kd)[e] = ka[k];

@@ -227,17 +227,20 @@ int pbsa_select_local(const pbsa_dims* dims, const float* scores, int nQB, int N
  *   pbsa_select_local(dims, scores, nQB, NB, win_ids, n_win, k, mem_ids, n_mem,
  *                     0, blk_len, mask, q_pos0, blk_pos, Tq, idx, cnt, Amax,
  *                     0, nQB)
- * with the same argument rules and limits.  The work runs as one cooperative
- * kernel (phases separated by grid barriers) when the shape has an
- * instantiation (n_win <= 256 and n_mem + min(k, n_win) <= 128) and a
- * co-resident grid; otherwise the call makes the three per-call launches
- * itself.
+ * with the same argument rules and limits.  The work runs as one persistent
+ * kernel when the shape has an instantiation (n_win <= 256 and n_mem +
+ * min(k, n_win) <= 128); otherwise the call makes the three per-call launches
+ * itself.  Inside the kernel every piece of work (a block to pool, a tile of
+ * scores, a head's update plan, a slot to write, eight attended lists) is a
+ * ticket handed out in order by an atomic counter, and each ticket waits
+ * (bounded in time) only for the per-head tickets it reads, so no step waits
+ * for every head of the step before it.
  *
  * workspace: device, 256-byte aligned, at least pbsa_route_workspace() bytes.
- * Its first 256 bytes hold the grid barrier's counters: zero them once before
- * the first call (e.g. cudaMemset); every call leaves them zero again.  The
- * rest is the update's workspace.  Calls that share a workspace must not run
- * concurrently.
+ * Its first C = 256 * ceil((16 + 20*B*H) / 256) bytes hold the kernel's
+ * counters: zero them once before the first call (e.g. cudaMemset); every
+ * call leaves them zero again.  The rest is the update's workspace.  Calls
+ * that share a workspace must not run concurrently.
  * ------------------------------------------------------------------------- */
 typedef struct {
   /* a1 + a2 */

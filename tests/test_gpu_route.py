@@ -2,8 +2,8 @@
 
 It must give, bit for bit, what the three per-call entry points give when made
 in order (pbsa_score_blocks -> pbsa_update_memory -> pbsa_select_local): both
-run the same device code, only the schedule differs (one cooperative kernel
-with grid barriers instead of five launches).  The per-call path is checked
+run the same device code, only the schedule differs (one persistent kernel
+whose work items wait on per-head counters instead of five launches).  The per-call path is checked
 against the oracle in test_gpu_parity.py; the fused path is also checked
 against the oracle directly on the decode snapshot.  The barrier words must be
 zero again after every call, and the call must work inside a CUDA graph.
@@ -39,8 +39,10 @@ def _same_state(La, Lb, where):
 
 
 def _barrier_words_zero(L):
+    # the kernel's counters: 4 control words and 5 per-(b,h) counters
     torch.cuda.synchronize()
-    assert int(L.rws[:16].count_nonzero()) == 0
+    n = 4 * (4 + 5 * L.w.B * L.w.H)
+    assert int(L.rws[:n].count_nonzero()) == 0
 
 
 def _snapshot_pair(name):
