@@ -521,41 +521,68 @@ def layer_bytes(L):
     return int(sum(t.numel() * t.element_size() for t in ts))
 
 
-def bench_rollouts(torch, timed_steps=6):
-    """Per-chunk latency of the rollout workloads (score -> update -> select ->
-    attend per layer) on device-drawn N(0,1) inputs, and their KV bytes."""
+def _pct(xs):
+    xs = np.asarray(xs, dtype=np.float64)
+    return {"mean": round(float(xs.mean()), 4), "p50": round(float(np.percentile(xs, 50)), 4),
+            "p90": round(float(np.percentile(xs, 90)), 4), "max": round(float(xs.max()), 4)}
+
+
+def _dense_attend(K, torch, d, q, Tc, pos0, kp, vp, NB, bl, bp, ids, nQB, o, lse, parts_o,
+                  parts_lse, max_list):
+    """Dense attention of a query chunk over the blocks `ids` with the library's
+    attention kernel; lists longer than the kernel's shared-memory list limit
+    run as parts whose outputs are merged by their log-sum-exps."""
+    parts = [ids[i:i + max_list] for i in range(0, len(ids), max_list)]
+    B, H = d.B, d.H
+    outs = []
+    for pi, part in enumerate(parts):
+        idx = part.expand(B, H, nQB, part.numel()).contiguous()
+        cnt = torch.full((B, H, nQB), part.numel(), dtype=torch.int32, device="cuda")
+        oo, ll = (o, lse) if len(parts) == 1 else (parts_o[pi], parts_lse[pi])
+        K.attn_fwd(d, q, Tc, pos0, kp, vp, NB, bl, bp, idx, cnt, part.numel(), 0, oo, ll)
+        outs.append((oo, ll))
+    if len(parts) > 1:
+        m = torch.stack([ll for _, ll in outs]).amax(0)
+        wsum = sum(torch.exp(ll - m) for _, ll in outs)
+        acc = sum(oo.float() * (torch.exp(ll - m) / wsum).unsqueeze(-1) for oo, ll in outs)
+        o.copy_(acc)
+        lse.copy_(m + torch.log(wsum))
+
+
+def bench_rollouts(torch):
+    """The rollout workloads as stated: every chunk step of the 20-second rollout
+    (27 steps, 1 layer) and of the 1-minute rollout (80 steps x 30 layers), each
+    step score -> update -> select -> attend per layer, on device-drawn seeded
+    inputs with the workloads' salience structure; per-step latency and its
+    percentiles; the same inputs through the library's attention kernel as the
+    dense comparators (every chunk so far, and the last W chunks); library KV
+    bytes against a dense cache, and the allocator's peak."""
     import pbsa_inputs as PI
+    from block_sparse_attention_39_b200 import pbsa as K
     from block_sparse_attention_39_b200.engine import PbsaLayer
     out = {}
-    g = torch.Generator(device="cuda").manual_seed(7)
     for name in ("rollout20s", "rollout1min"):
         w = PI.WORKLOADS[name]
+        torch.cuda.synchronize()
+        torch.cuda.empty_cache()
+        base = torch.cuda.memory_allocated()
+        torch.cuda.reset_peak_memory_stats()
         layers = [PbsaLayer(w) for _ in range(w.layers)]
-        shape = (w.B, w.H, w.chunk_tokens, w.D)
-        warm = 4
-        steps = warm + timed_steps
-        def draw():
-            return tuple(torch.randn(shape, generator=g, device="cuda").bfloat16() for _ in range(3))
-        # warm-up steps run eagerly; each timed step is a CUDA graph of every
-        # layer's score -> update -> select -> attend with the timing events
-        # inside it (so host launch overhead is not timed), replayed after the
-        # step's new chunk has been written
+        state_alloc = torch.cuda.memory_allocated() - base
         gs = torch.cuda.Stream()
-        times = []
-        for t in range(steps):
-            pre = [draw() for _ in layers]
+        pbsa_ms = []
+        for t in range(w.n_chunks):
             for li, L in enumerate(layers):
-                q, k, v = pre[li]
+                q, k, v = PI.chunk_tensors_device(w, t, li)
                 L.write_chunk(t, k, v)
                 L.q.copy_(q)
                 L.candidates(t)                 # id lists built outside the timed region
                 L.window_ids(t)
                 L.chunk_ids(t)
-            if t < warm:
-                for L in layers:
-                    L.step(t)
-                continue
+            del q, k, v
             torch.cuda.synchronize()
+            # each step: a CUDA graph of every layer's score -> update -> select ->
+            # attend with the timing events inside it (host launch cost not timed)
             ev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(2)]
             graph = torch.cuda.CUDAGraph()
             with torch.cuda.graph(graph, stream=gs):
@@ -566,18 +593,78 @@ def bench_rollouts(torch, timed_steps=6):
             with torch.cuda.stream(gs):
                 graph.replay()
             torch.cuda.synchronize()
-            times.append(tuple(ev))
+            pbsa_ms.append(ev[0].elapsed_time(ev[1]))
             del graph
-        torch.cuda.synchronize()
-        ms = float(np.mean([a.elapsed_time(b) for a, b in times]))
+        peak_alloc = torch.cuda.max_memory_allocated() - base
         kv = sum(layer_bytes(L) for L in layers)
-        dense_kv = w.n_chunks * layers[0].layout.nb_c * w.bs * w.D * 2 * 2 * w.B * w.H * w.layers
-        out[name] = {"layers": w.layers, "P": w.P, "policy": "merge_mean" if w.policy else "evict",
-                     "per_chunk_ms": round(ms, 4), "timed_steps": f"{warm}..{steps - 1}",
-                     "kv_bytes": kv, "dense_full_cache_kv_bytes_at_last_step": dense_kv,
-                     "kv_reduction": round(1 - kv / dense_kv, 4)}
-        del layers, pre
+        lay = layers[0].layout
+        nb_c = lay.nb_c
+        del layers
         torch.cuda.empty_cache()
+        # dense comparators: per layer a cache of every chunk so far, filled by
+        # pbsa_append_chunk with the same (layer, t) inputs; one layer's cache
+        # lives at a time, the per-step time is summed over the layers
+        NBd = w.n_chunks * nb_c
+        d = K.dims(w.B, w.H, w.D, w.bs, 1.0 / math.sqrt(w.D), torch.bfloat16)
+        dense_full = np.zeros(w.n_chunks)
+        dense_win = np.zeros(w.n_chunks)
+        max_list = 2048
+        Tc = w.chunk_tokens
+        kp = torch.zeros(w.B, w.H, NBd, w.bs, w.D, dtype=torch.bfloat16, device="cuda")
+        vp = torch.zeros_like(kp)
+        bl = torch.zeros(w.B, w.H, NBd, dtype=torch.int32, device="cuda")
+        bp = torch.zeros_like(bl)
+        kb = torch.zeros(w.B, w.H, NBd, w.D, dtype=torch.float32, device="cuda")
+        o = torch.empty(w.B, w.H, Tc, w.D, dtype=torch.bfloat16, device="cuda")
+        lse = torch.empty(w.B, w.H, Tc, dtype=torch.float32, device="cuda")
+        n_parts = -(-NBd // max_list)
+        parts_o = [torch.empty_like(o) for _ in range(n_parts)]
+        parts_lse = [torch.empty_like(lse) for _ in range(n_parts)]
+        all_ids = torch.arange(NBd, dtype=torch.int32, device="cuda")
+        dense_peak = 0
+        for li in range(w.layers):
+            bl.zero_()
+            for t in range(w.n_chunks):
+                q, k, v = PI.chunk_tensors_device(w, t, li)
+                blk = all_ids[t * nb_c:(t + 1) * nb_c]
+                K.append_chunk(d, k, v, Tc, t * Tc, kp, vp, NBd, blk, bl, bp, kb)
+                for kind, ids in (("full", all_ids[:(t + 1) * nb_c]),
+                                  ("win", all_ids[max(0, t + 1 - w.W) * nb_c:(t + 1) * nb_c])):
+                    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    e0.record()
+                    _dense_attend(K, torch, d, q, Tc, t * Tc, kp, vp, NBd, bl, bp, ids, nb_c, o,
+                                  lse, parts_o, parts_lse, max_list)
+                    e1.record()
+                    torch.cuda.synchronize()
+                    (dense_full if kind == "full" else dense_win)[t] += e0.elapsed_time(e1)
+            dense_peak = max(dense_peak, torch.cuda.max_memory_allocated() - base)
+        dense_kv_last = NBd * w.bs * w.D * 2 * 2 * w.B * w.H * w.layers
+        del kp, vp, bl, bp, kb, o, lse, parts_o, parts_lse
+        torch.cuda.empty_cache()
+        pb = np.array(pbsa_ms)
+        out[name] = {
+            "layers": w.layers, "P": w.P, "policy": "merge_mean" if w.policy else "evict",
+            "steps": w.n_chunks,
+            "inputs": "device-drawn per (layer, step), N(0,1) with the workload's salient blocks "
+                      "(N(0,2) offsets), the same draws for PBSA and the dense comparators",
+            "pbsa_ms_per_step": _pct(pb),
+            "pbsa_ms_steps": [round(float(x), 4) for x in pb],
+            "dense_full_cache_ms_per_step": _pct(dense_full),
+            "dense_full_cache_ms_steps": [round(float(x), 4) for x in dense_full],
+            "dense_sliding_window_ms_per_step": _pct(dense_win),
+            "speedup_vs_dense_full_cache": {
+                "whole_rollout": round(float(dense_full.sum() / pb.sum()), 3),
+                "last_step": round(float(dense_full[-1] / pb[-1]), 3)},
+            "kv_bytes_library": kv,
+            "allocator_bytes_pbsa_state": int(state_alloc),
+            "allocator_peak_bytes_pbsa_rollout": int(peak_alloc),
+            "dense_full_cache_kv_bytes_at_last_step": dense_kv_last,
+            "allocator_peak_bytes_dense_one_layer": int(dense_peak),
+            "kv_reduction": round(1 - kv / dense_kv_last, 4),
+            "dense_note": "PBSA step = score + update + select + attend per layer; dense = the "
+                          "attention kernel over every chunk so far (lists over 2048 blocks run "
+                          "as parts merged by log-sum-exp) or the last W chunks; per step summed "
+                          "over the layers"}
     return out
 
 

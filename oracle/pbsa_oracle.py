@@ -22,7 +22,10 @@ step in plain float64 numpy with Python loops over (batch, head, block):
 * a6     hybrid attention: dense over the persistent memory, sparse over the
          local window (section 2 PBSA, item "Atención Híbrida");
 * a7     the backward pass of a6 for the trainable path (section 3
-         "Contribuciones Clave", item "Kernel PBSA"; section 2 "Entrenamiento").
+         "Contribuciones Clave", item "Kernel PBSA"; section 2 "Entrenamiento");
+* the backward of a3 and the recurrent backward of a rollout, through the
+         slots a block was copied or merged into (section 2 "Entrenamiento";
+         the abstract).
 
 The pages give no formulas.  Where they are silent this module takes the
 plainest reading; each reading is named in the docstring of the function that
@@ -223,7 +226,11 @@ def update_memory(kpool, vpool, blk_len, blk_pos, k_bar, slot_src, slot_w,
     [B,H,NB].  ``store`` is the storage type new slot rows are rounded to.
 
     Returns (kpool, vpool, blk_len, blk_pos, k_bar, slot_src, slot_w, info) with
-    ``info[(b,h)] = dict(kept=[src...], losers=[src...], target={src: slot})``.
+    ``info[(b,h)] = dict(kept=[src...], losers=[src...], target={src: slot},
+    compose={slot: [(pre-update id, weight, rows), ...]})``: every slot after
+    the update is the weighted row-wise sum of those terms (a copy is one term
+    of weight 1 over the whole block; an emptied slot has none), before the
+    rounding to the storage type.
     """
     kp = np.array(kpool, dtype=np.float64, copy=True)
     vp = np.array(vpool, dtype=np.float64, copy=True)
@@ -284,8 +291,14 @@ def update_memory(kpool, vpool, blk_len, blk_pos, k_bar, slot_src, slot_w,
                           int(ps[b, h, c]), kb[b, h, c].copy()) for s, c in sinks_in}
 
             holder = {slot_of[id(it)]: it for it in kept}
+            bs = kp.shape[3]
+            # what each slot holds after the update, as (pre-update id, weight,
+            # rows) terms of a weighted row-wise mean: the backward of the
+            # update distributes a slot's gradient by these terms (NEXT-2)
+            compose = {s: [(s, 1.0, bs)] for s in range(n_sink)}
             for s in range(n_sink, P):
                 if s not in holder:
+                    compose[s] = []
                     ss[b, h, s] = -1
                     sw[b, h, s] = 0.0
                     ln[b, h, s] = 0
@@ -295,6 +308,7 @@ def update_memory(kpool, vpool, blk_len, blk_pos, k_bar, slot_src, slot_w,
                 c = holder[s]
                 group = merged_into[s]
                 if not group:
+                    compose[s] = [(c.phys, 1.0, bs)]
                     kp[b, h, s] = K[id(c)]
                     vp[b, h, s] = V[id(c)]
                     ln[b, h, s] = L[id(c)]
@@ -302,6 +316,8 @@ def update_memory(kpool, vpool, blk_len, blk_pos, k_bar, slot_src, slot_w,
                     sw[b, h, s] = c.w
                 else:
                     W = c.w + sum(j.w for j in group)
+                    compose[s] = [(c.phys, c.w / W, L[id(c)])] + \
+                        [(j.phys, j.w / W, L[id(j)]) for j in group]
                     ksum = c.w * _masked_rows(K[id(c)], L[id(c)])
                     vsum = c.w * _masked_rows(V[id(c)], L[id(c)])
                     for j in group:
@@ -316,13 +332,15 @@ def update_memory(kpool, vpool, blk_len, blk_pos, k_bar, slot_src, slot_w,
                 ss[b, h, s] = c.src
                 ps[b, h, s] = POS[id(c)]
             for s, (k_, v_, l_, p_, kb_) in sink_K.items():
+                compose[s] = [(dict(sinks_in)[s], 1.0, bs)]
                 kp[b, h, s], vp[b, h, s] = k_, v_
                 ln[b, h, s], ps[b, h, s], kb[b, h, s] = l_, p_, kb_
                 ss[b, h, s] = s
                 sw[b, h, s] = 1.0
             info[(b, h)] = dict(kept=[it.src for it in kept], losers=[it.src for it in losers],
                                 keys={it.src: it.m for it in items}, target=target,
-                                slot={it.src: slot_of[id(it)] for it in kept})
+                                slot={it.src: slot_of[id(it)] for it in kept},
+                                compose=compose)
     return kp, vp, ln, ps, kb, ss, sw, info
 
 
@@ -507,6 +525,84 @@ def attention_bwd(q, kpool, vpool, blk_len, blk_pos, idx, cnt, dO, scale: float,
                     dv[b, h, j, :m] += dvc[off:off + m]
                     off += m
     return dq, dk, dv
+
+
+# ---------------------------------------------------------------------------
+# NEXT-2  the recurrent trainable path: gradients through the memory update
+# ---------------------------------------------------------------------------
+
+def update_memory_vjp(dk_after, dv_after, info, P: int):
+    """Backward of ``update_memory`` for the key and value rows.
+
+    Sparse Forcing trains with the dynamically updated cache, and its memory
+    learns to compress, keep and refresh persistent blocks (gist.science/es,
+    section 2 "Entrenamiento"; the abstract on the shd-paper.top page), so the
+    loss reaches a block's keys and values also through the slots it was
+    copied or merged into.  Every slot after the update is a weighted row-wise
+    sum of pre-update blocks (``info[(b,h)]["compose"]``, R5: rows past a
+    block's length count as zero; the rounding to storage is taken as the
+    identity), so the vector-Jacobian product is that sum transposed:
+
+        d(pre id j)[r] += weight * d(slot s)[r]   for r < rows, every term (j,
+        weight, rows) of slot s;
+
+    blocks that are not slots keep their own gradient (the update reads them
+    only), and a pre-update slot gets only what reaches it through the terms.
+    The selection and merge decisions are constants (R13).
+
+    dk_after / dv_after: [B,H,NB,bs,D] gradients w.r.t. the pool after the
+    update.  Returns the gradients w.r.t. the pool before it."""
+    dk = np.array(dk_after, dtype=np.float64, copy=True)
+    dv = np.array(dv_after, dtype=np.float64, copy=True)
+    dk[:, :, :P] = 0.0
+    dv[:, :, :P] = 0.0
+    for (b, h), inf in info.items():
+        for s, terms in inf["compose"].items():
+            for j, wgt, n in terms:
+                dk[b, h, j, :n] += wgt * dk_after[b, h, s, :n]
+                dv[b, h, j, :n] += wgt * dv_after[b, h, s, :n]
+    return dk, dv
+
+
+def rollout_bwd(steps, P: int, place, W: int, T_c: int, scale: float, mask: int = MASK_CHUNK):
+    """Gradients of a rollout's loss sum_t <O_t, dO_t> w.r.t. every chunk's
+    queries, keys and values, through the attention of each step and through
+    the persistent memory (the recurrent trainable path).
+
+    ``steps[t]`` holds what step t of the forward used: q [B,H,T_c,D], the
+    pool after its memory update (kp, vp, bl, bp), its lists (idx, cnt), the
+    update's ``info`` (None if no update ran) and dO.  Going back in time, the
+    gradient of the slots after update t is what attention t gives them plus
+    what the later steps pass back to the slots before update t+1; the
+    update's backward (``update_memory_vjp``) then hands the slots' gradient
+    to the blocks they came from.  Before update t the ring holds chunks
+    t-W .. t (``place``); a ring block's gradient belongs to the chunk in it.
+
+    Returns (dq, dk, dv): lists over t of [B,H,T_c,D] (dq for step t's
+    queries; dk, dv for chunk t's keys and values)."""
+    T = len(steps)
+    B, H, NB, bs, D = steps[0]["kp"].shape
+    Gk = np.zeros((B, H, P, bs, D))
+    Gv = np.zeros((B, H, P, bs, D))
+    dq = [None] * T
+    dkc = [np.zeros((B, H, T_c, D)) for _ in range(T)]
+    dvc = [np.zeros((B, H, T_c, D)) for _ in range(T)]
+    for t in reversed(range(T)):
+        st = steps[t]
+        dq[t], dk, dv = attention_bwd(st["q"], st["kp"], st["vp"], st["bl"], st["bp"],
+                                      st["idx"], st["cnt"], st["dO"], scale, mask, t * T_c)
+        if P:
+            dk[:, :, :P] += Gk
+            dv[:, :, :P] += Gv
+        if st["info"] is not None:
+            dk, dv = update_memory_vjp(dk, dv, st["info"], P)
+        if P:
+            Gk, Gv = dk[:, :, :P].copy(), dv[:, :, :P].copy()
+        for c in range(max(0, t - W), t + 1):
+            for pid, (r0, n) in zip(place.chunk_ids(c), place.blocks):
+                dkc[c][:, :, r0:r0 + n] += dk[:, :, pid, :n]
+                dvc[c][:, :, r0:r0 + n] += dv[:, :, pid, :n]
+    return dq, dkc, dvc
 
 
 # ---------------------------------------------------------------------------

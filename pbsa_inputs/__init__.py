@@ -167,3 +167,30 @@ def snapshot_chunks(w: Workload, layer: int = 0):
 
 def grad_output(w: Workload, T: int, layer: int = 0) -> np.ndarray:
     return round_to_storage(normal((w.B, w.H, T, w.D), w.seed, "do", layer), w.dtype)
+
+
+def chunk_tensors_device(w: Workload, t: int, layer: int = 0, device: str = "cuda"):
+    """Q, K, V of chunk ``t`` as bf16 device tensors [B, H, chunk_tokens, D]
+    drawn on the device from a generator keyed by (workload seed, layer, t),
+    with the salience structure of ``chunk_tensors`` (the same salient runs;
+    offsets drawn on the device).  Same distributions as ``chunk_tensors``,
+    other values: for timing runs too large to draw on the host, where both
+    sides of a comparison draw the same (layer, t) from this function."""
+    import torch
+    h = hashlib.sha256(repr((w.seed, "device", layer, t)).encode()).digest()
+    g = torch.Generator(device=device).manual_seed(int.from_bytes(h[:8], "little") >> 1)
+    shape = (w.B, w.H, w.chunk_tokens, w.D)
+    q = torch.randn(shape, generator=g, device=device)
+    k = torch.randn(shape, generator=g, device=device)
+    v = torch.randn(shape, generator=g, device=device)
+    runs = -(-w.chunk_tokens // w.bs)
+    if w.salient_frac > 0:
+        if w.salient_scope == "chunk":
+            sal = _salient_runs(w, layer, runs, ("chunk", t // w.redraw_every))
+        else:
+            sal_all = _salient_runs(w, layer, w.n_chunks * runs, ("cache",))
+            sal = [j - t * runs for j in sal_all if t * runs <= j < (t + 1) * runs]
+        for j in sal:
+            off = math.sqrt(2.0) * torch.randn((w.B, w.H, 1, w.D), generator=g, device=device)
+            k[:, :, j * w.bs:(j + 1) * w.bs, :] += off
+    return q.bfloat16(), k.bfloat16(), v.bfloat16()
