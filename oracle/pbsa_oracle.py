@@ -400,6 +400,79 @@ def select_local(S: np.ndarray, win_ids, k: int, mem_ids: Optional[np.ndarray],
     return out
 
 
+def frame_groups(T_c: int, bs: int, frame_tokens: int):
+    """The frame of each block of a chunk (R20): block j (rows [j*bs, ...) of the
+    chunk) belongs to the frame its first row falls in, frame_tokens rows per
+    frame.  Returns a list over the chunk's blocks."""
+    return [(r0 // frame_tokens) for r0, _ in chunk_blocks(T_c, bs)]
+
+
+def _frame_scores(cands, s_row, lens):
+    """R20: {frame: sum_j len_j s_j / sum_j len_j} over the (block, frame) pairs."""
+    num, den = {}, {}
+    for j, g in cands:
+        num[g] = num.get(g, 0.0) + float(lens[j]) * float(s_row[j])
+        den[g] = den.get(g, 0.0) + float(lens[j])
+    return {g: num[g] / den[g] for g in num}
+
+
+def select_hier(S: np.ndarray, win_ids, win_frame, F: int, k: int,
+                mem_ids: Optional[np.ndarray], blk_len: np.ndarray, mask: int = MASK_CHUNK,
+                q_pos0: int = 0, blk_pos: Optional[np.ndarray] = None, bs: int = 0,
+                Tq: int = 0, q_chunk: int = 0):
+    """Two-level local selection, frame then block, the alternative router of
+    the "next" rows (Light Forcing, gist.science/it, section 2.2 "Attenzione
+    Sparsa Gerarchica (HSA)": query and key tokens are mean-pooled per block
+    and per frame; each query block first keeps a few relevant historical
+    frames by their frame-level keys, then the critical blocks inside those
+    frames by their block-level keys; attention runs over the kept blocks).
+
+    Readings taken:
+      R20  a frame of the window is the group of window blocks that start in it
+           (``win_frame[e]`` is the frame of window entry e, any integer label);
+           its pooled key is the mean of its blocks' valid tokens, so its score
+           for query block i is the length-weighted mean of those blocks'
+           scores: sum_j len_j S_ij / sum_j len_j, over the blocks that are
+           candidates for i (length > 0 and, with the token mask, allowed);
+      R21  the F frames of highest score are kept (ties: lower frame label);
+           the local set is the Top-K blocks of the kept frames by S (ties:
+           lower id), all of them if fewer; the list is the union with the
+           memory as in ``select_local``.
+    With F at least the number of frames this is ``select_local``.
+
+    Shapes and the other arguments as ``select_local``.  Returns A[b][h][i]."""
+    B, H, nQB, _ = S.shape
+    blocks = query_blocks(Tq, bs, q_chunk) if mask == MASK_TOKEN else None
+    out = []
+    for b in range(B):
+        ob = []
+        for h in range(H):
+            oh = []
+            mem = []
+            if mem_ids is not None:
+                mem = [int(m) for m in mem_ids[b, h] if m >= 0 and blk_len[b, h, m] > 0]
+            for i in range(nQB):
+                cands = []
+                for j, g in zip(win_ids, win_frame):
+                    j = int(j)
+                    if blk_len[b, h, j] <= 0:
+                        continue
+                    if mask == MASK_TOKEN:
+                        last_q = q_pos0 + blocks[i][0] + blocks[i][1] - 1
+                        if blk_pos[b, h, j] > last_q:
+                            continue
+                    cands.append((j, int(g)))
+                fs = _frame_scores(cands, S[b, h, i], blk_len[b, h])
+                frames = sorted(fs, key=lambda g: (-fs[g], g))[:max(F, 0)]
+                kept = set(frames)
+                order = sorted([j for j, g in cands if g in kept], key=lambda j: (-S[b, h, i, j], j))
+                local = order[:min(k, len(order))]
+                oh.append(sorted(set(mem) | set(local)))
+            ob.append(oh)
+        out.append(ob)
+    return out
+
+
 def lists_to_arrays(A, Amax: int):
     """Pack attended lists into idx [B,H,nQB,Amax] (padding -1) and cnt [B,H,nQB]."""
     B, H, nQB = len(A), len(A[0]), len(A[0][0])
