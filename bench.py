@@ -600,7 +600,10 @@ def bench_rollouts(torch):
         lay = layers[0].layout
         nb_c = lay.nb_c
         del layers
+        torch.cuda.synchronize()
         torch.cuda.empty_cache()
+        base = torch.cuda.memory_allocated()
+        torch.cuda.reset_peak_memory_stats()
         # dense comparators: per layer a cache of every chunk so far, filled by
         # pbsa_append_chunk with the same (layer, t) inputs; one layer's cache
         # lives at a time, the per-step time is summed over the layers

@@ -48,9 +48,17 @@ SIGNATURES = {
     "pbsa_update_memory": (c_int, [P, c_void_p, c_void_p, c_int, c_void_p, c_void_p, c_void_p,
                                    c_int, c_int, c_void_p, c_void_p, c_void_p, c_void_p, c_int,
                                    c_void_p, c_int, c_void_p, c_size_t, c_void_p]),
+    "pbsa_update_plan_bytes": (c_size_t, [P, c_int, c_int]),
+    "pbsa_update_memory_bwd_workspace": (c_size_t, [P, c_int]),
+    "pbsa_update_memory_bwd": (c_int, [P, c_int, c_int, c_int, c_void_p, c_void_p, c_void_p,
+                                       c_void_p, c_size_t, c_void_p]),
     "pbsa_select_local": (c_int, [P, c_void_p, c_int, c_int, c_void_p, c_int, c_int, c_void_p,
                                   c_int, c_int, c_void_p, c_int, c_int, c_void_p, c_int, c_void_p,
                                   c_void_p, c_int, c_int, c_int, c_void_p]),
+    "pbsa_select_hier": (c_int, [P, c_void_p, c_int, c_int, c_void_p, c_void_p, c_int, c_int,
+                                 c_int, c_int, c_void_p, c_int, c_int, c_void_p, c_int, c_int,
+                                 c_void_p, c_int, c_void_p, c_void_p, c_int, c_int, c_int,
+                                 c_void_p]),
     "pbsa_route_workspace": (c_size_t, [P, c_int, c_int]),
     "pbsa_route_step": (c_int, [P, ctypes.POINTER(PbsaRouteArgs), c_void_p, c_size_t, c_void_p]),
     "pbsa_attn_fwd": (c_int, [P, c_void_p, c_int, c_int, c_void_p, c_void_p, c_int, c_void_p,

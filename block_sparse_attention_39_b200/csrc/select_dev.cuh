@@ -363,5 +363,162 @@ __device__ __forceinline__ void select_row_bitmap(const SelArgs& a, int i, long 
   SEL_TRACE(i, bh, 5);
 }
 
+// Shared memory per warp of select_row_hier: that of select_row_bitmap plus
+// the window's per-entry (weighted score, length, frame) for the frame scores.
+template <int W>
+__host__ __device__ constexpr int sel_hier_smem_per_warp() {
+  return sel_bitmap_smem_per_warp<W>() + 32 * W * 12;
+}
+
+// The two-level local selection (frame, then block) for query block i of head
+// bh, computed by one warp; the list is the union with the memory ids as in
+// select_row.  Light Forcing keeps, per query block, a few relevant frames by
+// frame-level pooled keys and then the critical blocks inside them by
+// block-level keys (gist.science/it, section 2.2 "Attenzione Sparsa
+// Gerarchica (HSA)").  Here a frame is a group of window blocks (win_frame[e]
+// is the frame of window entry e, 0 <= label < n_frames <= 32); its score is
+// the length-weighted mean of its candidate blocks' scores (its pooled key is
+// the mean of its blocks' tokens and scores are linear in the key), summed in
+// window order; the F frames of highest score are kept (ties: lower label) and
+// the Top-K blocks of the kept frames are taken as in select_row_bitmap.
+template <int W, int U>
+__device__ __forceinline__ void select_row_hier(const SelArgs& a, const int32_t* win_frame,
+                                                int n_frames, int F, int i, long bh,
+                                                uint8_t* wsm) {
+  uint64_t* skeys = reinterpret_cast<uint64_t*>(wsm);                 // [32*W]
+  uint32_t* bm = reinterpret_cast<uint32_t*>(wsm + 32 * W * 8);       // [kSelBmWords]
+  float* f_num = reinterpret_cast<float*>(wsm + sel_bitmap_smem_per_warp<W>());  // [32*W]
+  float* f_den = f_num + 32 * W;                                      // [32*W]
+  int* f_lab = reinterpret_cast<int*>(f_den + 32 * W);                // [32*W]
+  const int NB = a.NB, n_win = a.n_win, n_mem = a.n_mem;
+  const int lane = threadIdx.x & 31;
+  const float* srow = a.scores + (bh * a.nQB_total + a.qb_offset + i) * static_cast<long>(NB);
+  int qrow0, qlen;
+  qb_rows(i, a.Tq, a.qc, a.bs, qrow0, qlen);
+  const int last_q = a.q_pos0 + qrow0 + qlen - 1;
+  const int nbw = (NB + 31) / 32;
+
+  int wid[W], wfr[W], mid[U];
+#pragma unroll
+  for (int r = 0; r < W; ++r) {
+    const int e = lane + 32 * r;
+    wid[r] = e < n_win ? a.win_ids[e] : -1;
+    wfr[r] = e < n_win ? win_frame[e] : -1;
+  }
+#pragma unroll
+  for (int r = 0; r < U; ++r) {
+    const int me = lane + 32 * r;
+    mid[r] = me < n_mem ? a.mem_ids[bh * a.mem_ld + me] : -1;
+  }
+  for (int w = lane; w < nbw; w += 32) bm[w] = 0u;
+  // ---- candidates of the window, and their frames' weighted scores
+  uint64_t wkey[W];
+#pragma unroll
+  for (int r = 0; r < W; ++r) {
+    const int j = wid[r];
+    const int e = lane + 32 * r;
+    const bool in = j >= 0 && j < NB;
+    if (e < n_win && !in) report_status(a.status, PBSA_ERR_ARG);
+    const bool lab_ok = wfr[r] >= 0 && wfr[r] < n_frames;
+    if (e < n_win && !lab_ok) report_status(a.status, PBSA_ERR_ARG);
+    const int len = in ? sel_len(a, bh, j) : 0;
+    const float sc = in ? srow[j] : 0.f;
+    const int pos = (in && a.mask == PBSA_MASK_TOKEN) ? sel_pos(a, bh, j) : 0;
+    bool ok = len > 0 && lab_ok;
+    if (a.mask == PBSA_MASK_TOKEN) ok = ok && pos <= last_q;
+    wkey[r] = ok ? score_key(sc, static_cast<uint32_t>(j)) : 0ull;
+    f_num[e] = ok ? static_cast<float>(len) * sc : 0.f;
+    f_den[e] = ok ? static_cast<float>(len) : 0.f;
+    f_lab[e] = ok ? wfr[r] : -1;
+  }
+  __syncwarp();
+  // lane g sums frame g over the window in order
+  float num = 0.f, den = 0.f;
+  if (lane < n_frames) {
+    for (int e = 0; e < n_win; ++e) {
+      if (f_lab[e] == lane) {
+        num += f_num[e];
+        den += f_den[e];
+      }
+    }
+  }
+  const bool has = den > 0.f;
+  const float fs = has ? num / den : -INFINITY;
+  int frank = 0;
+#pragma unroll 4
+  for (int m = 0; m < 32; ++m) {
+    const float o = __shfl_sync(0xffffffffu, fs, m);
+    const bool oh = __shfl_sync(0xffffffffu, has, m);
+    frank += (oh && (o > fs || (o == fs && m < lane))) ? 1 : 0;
+  }
+  const uint32_t kept = __ballot_sync(0xffffffffu, lane < n_frames && has && frank < F);
+  // ---- Top-K of the kept frames' blocks by counting rank
+  int n_ok = 0;
+#pragma unroll
+  for (int r = 0; r < W; ++r) {
+    if (wkey[r] != 0ull && !((kept >> wfr[r]) & 1u)) wkey[r] = 0ull;
+    skeys[lane + 32 * r] = wkey[r];
+    n_ok += __popc(__ballot_sync(0xffffffffu, wkey[r] != 0ull));
+  }
+  __syncwarp();
+  const int take = min(a.k, n_ok);
+  int rank[W];
+#pragma unroll
+  for (int r = 0; r < W; ++r) rank[r] = 0;
+  const ulonglong2* k2 = reinterpret_cast<const ulonglong2*>(skeys);
+#pragma unroll 4
+  for (int f = 0; f < 16 * W; ++f) {
+    const ulonglong2 v = k2[f];
+#pragma unroll
+    for (int r = 0; r < W; ++r) rank[r] += (v.x > wkey[r] ? 1 : 0) + (v.y > wkey[r] ? 1 : 0);
+  }
+#pragma unroll
+  for (int r = 0; r < W; ++r)
+    if (wkey[r] != 0ull && rank[r] < take) atomicOr(&bm[wid[r] >> 5], 1u << (wid[r] & 31));
+#pragma unroll
+  for (int r = 0; r < U; ++r) {
+    const int m = mid[r];
+    if (m >= NB || m < -1) report_status(a.status, PBSA_ERR_ARG);
+    if (m >= 0 && m < NB && sel_len(a, bh, m) > 0) atomicOr(&bm[m >> 5], 1u << (m & 31));
+  }
+  __syncwarp();
+  int total = 0;
+  for (int w0 = 0; w0 < nbw; w0 += 32) {
+    const uint32_t word = w0 + lane < nbw ? bm[w0 + lane] : 0u;
+    int c = __popc(word);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) c += __shfl_xor_sync(0xffffffffu, c, off);
+    total += c;
+  }
+  int32_t* out = a.idx + (bh * a.nQB_total + a.qb_offset + i) * static_cast<long>(a.Amax);
+  int32_t* cnt = a.cnt + bh * a.nQB_total + a.qb_offset + i;
+  if (total > a.Amax) {
+    if (lane == 0) report_status(a.status, PBSA_ERR_SHAPE);
+    for (int e = lane; e < a.Amax; e += 32) out[e] = -1;
+    if (lane == 0) *cnt = 0;
+    return;
+  }
+  int base = 0;
+  for (int w0 = 0; w0 < nbw; w0 += 32) {
+    uint32_t word = w0 + lane < nbw ? bm[w0 + lane] : 0u;
+    const int c = __popc(word);
+    int incl = c;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += v;
+    }
+    int pos = base + incl - c;
+    while (word) {
+      const int b = __ffs(word) - 1;
+      out[pos++] = (w0 + lane) * 32 + b;
+      word &= word - 1u;
+    }
+    base += __shfl_sync(0xffffffffu, incl, 31);
+  }
+  for (int e = total + lane; e < a.Amax; e += 32) out[e] = -1;
+  if (lane == 0) *cnt = total;
+}
+
 }  // namespace dev
 }  // namespace pbsa

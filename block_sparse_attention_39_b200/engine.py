@@ -158,6 +158,30 @@ class PbsaLayer:
                        self.blk_pos, w.chunk_tokens, self.idx, self.cnt, self.Amax, 0, self.nQB,
                        stream)
 
+    def frame_labels(self, t, frame_tokens):
+        """Frame of each window entry (window order) for the two-level selection:
+        the window's chunks in order, each cut into frames of frame_tokens rows;
+        a block belongs to the frame its first row falls in.  Returns (labels on
+        the device, number of frames)."""
+        lay = self.layout
+        chunks = lay.window_chunks(t)
+        per = -(-lay.chunk_tokens // frame_tokens)
+        labels = [ci * per + (j * lay.bs) // frame_tokens
+                  for ci in range(len(chunks)) for j in range(lay.nb_c)]
+        return self.ids(("frames", len(chunks), frame_tokens), labels), len(chunks) * per
+
+    def select_hier(self, t, F, frame_tokens, stream=None):
+        """The two-level local selection (frames of frame_tokens rows, the best F of
+        them, then the top-k blocks inside) united with the memory
+        (pbsa_select_hier); writes self.idx / self.cnt like select()."""
+        w = self.w
+        win = self.window_ids(t)
+        labels, n_frames = self.frame_labels(t, frame_tokens)
+        K.select_hier(self.d, self.scores, self.nQB, self.NB, win, labels, win.numel(), n_frames,
+                      F, w.k, self.mem_ids, self.P, self.blk_len, w.mask, t * w.chunk_tokens,
+                      self.blk_pos, w.chunk_tokens, self.idx, self.cnt, self.Amax, 0, self.nQB,
+                      stream)
+
     def attend(self, t, stream=None):
         w = self.w
         if self.tdtype == torch.bfloat16:
@@ -334,3 +358,79 @@ class PbsaTrain:
         K.attn_bwd(self.d, self.q, self.T, 0, self.kpool, self.vpool, self.NB, self.blk_len,
                    self.blk_pos, self.idx, self.cnt, self.Amax, self.w.mask, self.o, self.lse,
                    self.dO, self.dq, self.dk, self.dv, self.ws, stream)
+
+
+class PbsaRolloutTrain:
+    """The recurrent trainable path of a rollout (Sparse Forcing trains with
+    the dynamically updated cache): the chunk steps of a ``PbsaLayer`` run
+    forward with each step recorded -- its queries, the pool after its memory
+    update, its lists, outputs and the update's plan -- and then the backward
+    of the loss sum_t <O_t, dO_t> back in time: the attention backward of step
+    t (pbsa_attn_bwd) gives the gradient of every pool block it read; the slots
+    also receive what the later steps pass back; the memory update's backward
+    (pbsa_update_memory_bwd) hands the slots' gradient to the blocks they were
+    copied or merged from.  A ring block's gradient belongs to the chunk held
+    at that ring position.  Selections and merges are constants."""
+
+    def __init__(self, layer: PbsaLayer):
+        self.L = L = layer
+        w = L.w
+        self.steps = []
+        self.plan_bytes = K.update_plan_bytes(L.d, L.P, L.max_cand) if L.P else 0
+        self.bwd_ws = torch.empty(K.attn_bwd_workspace(L.dbf, w.chunk_tokens, L.NB, L.Amax),
+                                  dtype=torch.uint8, device=L.dev)
+        self.upd_ws = (torch.empty(K.update_memory_bwd_workspace(L.d, L.P), dtype=torch.uint8,
+                                   device=L.dev) if L.P else None)
+
+    def step(self, t, q, k, v, stream=None):
+        """Chunk t's Q/K/V [B,H,T_c,D] (the layer's storage type) through
+        score -> update -> select -> attend, recorded for the backward."""
+        L = self.L
+        L.write_chunk(t, k, v)
+        L.q.copy_(q)
+        L.score(t, stream=stream)
+        ci, cs = L.candidates(t)
+        L.update(ci, cs, stream=stream)
+        L.select(t, stream=stream)
+        L.attend(t, stream=stream)
+        n_cand = ci.numel() if L.P else 0
+        self.steps.append(dict(
+            q=L.q.clone(), kpool=L.kpool.clone(), vpool=L.vpool.clone(),
+            blk_len=L.blk_len.clone(), blk_pos=L.blk_pos.clone(), idx=L.idx.clone(),
+            cnt=L.cnt.clone(), o=L.o.clone(), lse=L.lse.clone(), n_cand=n_cand,
+            plan=L.ws[:self.plan_bytes].clone() if n_cand else None))
+        return L.o, L.lse
+
+    def backward(self, dOs, stream=None):
+        """dOs: dO [B,H,T_c,D] (bf16) of every recorded step.  Returns (dq, dk,
+        dv): float32 [B,H,T_c,D] per step (dq) and per chunk (dk, dv)."""
+        L, w = self.L, self.L.w
+        lay = L.layout
+        T, P, Tc = len(self.steps), L.P, w.chunk_tokens
+        shape = (w.B, w.H, Tc, w.D)
+        f32 = dict(dtype=torch.float32, device=L.dev)
+        dq = [torch.empty(shape, **f32) for _ in range(T)]
+        dkc = [torch.zeros(shape, **f32) for _ in range(T)]
+        dvc = [torch.zeros(shape, **f32) for _ in range(T)]
+        dk = torch.empty(w.B, w.H, L.NB, w.bs, w.D, **f32)
+        dv = torch.empty_like(dk)
+        Gk = Gv = None
+        for t in reversed(range(T)):
+            r = self.steps[t]
+            K.attn_bwd(L.dbf, r["q"], Tc, t * Tc, r["kpool"], r["vpool"], L.NB, r["blk_len"],
+                       r["blk_pos"], r["idx"], r["cnt"], L.Amax, w.mask, r["o"], r["lse"],
+                       dOs[t], dq[t], dk, dv, self.bwd_ws, stream)
+            if P:
+                if Gk is not None:
+                    dk[:, :, :P] += Gk
+                    dv[:, :, :P] += Gv
+                if r["plan"] is not None:
+                    K.update_memory_bwd(L.d, L.NB, P, r["n_cand"], r["plan"], dk, dv,
+                                        self.upd_ws, stream)
+                Gk, Gv = dk[:, :, :P].clone(), dv[:, :, :P].clone()
+            for c in range(max(0, t - w.W), t + 1):
+                ids = torch.as_tensor(lay.chunk_phys_ids(c), dtype=torch.long, device=L.dev)
+                # a chunk's blocks tile its rows in order, only the last one partial
+                dkc[c] += dk[:, :, ids].reshape(w.B, w.H, -1, w.D)[:, :, :Tc]
+                dvc[c] += dv[:, :, ids].reshape(w.B, w.H, -1, w.D)[:, :, :Tc]
+        return dq, dkc, dvc

@@ -84,6 +84,24 @@ def update_memory(d: PbsaDims, kpool, vpool, NB, blk_len, blk_pos, k_bar, P, n_s
         _p(workspace), workspace.numel() * workspace.element_size(), _s(stream)))
 
 
+def update_plan_bytes(d: PbsaDims, P: int, n_cand: int) -> int:
+    """Bytes at the head of the update workspace that hold the step's plan
+    (what pbsa_update_memory_bwd reads)."""
+    return int(lib().pbsa_update_plan_bytes(ctypes.byref(d), P, n_cand))
+
+
+def update_memory_bwd_workspace(d: PbsaDims, P: int) -> int:
+    return int(lib().pbsa_update_memory_bwd_workspace(ctypes.byref(d), P))
+
+
+def update_memory_bwd(d: PbsaDims, NB, P, n_cand, plan, dk, dv, workspace, stream=None):
+    """pbsa_update_memory_bwd: dk / dv (float, pool-shaped) go from the gradient
+    w.r.t. the pool after the update to the gradient w.r.t. the pool before it."""
+    _check("pbsa_update_memory_bwd", lib().pbsa_update_memory_bwd(
+        ctypes.byref(d), NB, P, n_cand, _p(plan), _p(dk), _p(dv), _p(workspace),
+        workspace.numel() * workspace.element_size(), _s(stream)))
+
+
 def select_local(d: PbsaDims, scores, nQB, NB, win_ids, n_win, k, mem_ids, n_mem, blk_len, mask,
                  q_pos0, blk_pos, Tq, idx, cnt, Amax, qb_offset=0, nQB_total=None, stream=None,
                  mem_ld=0, mem_offset=0):
@@ -98,6 +116,16 @@ def select_local(d: PbsaDims, scores, nQB, NB, win_ids, n_win, k, mem_ids, n_mem
         ctypes.byref(d), _p(scores), nQB, NB, _p(win_ids), n_win, k, mp, n_mem, mem_ld,
         _p(blk_len), mask, q_pos0, _p(blk_pos), Tq, _p(idx), _p(cnt), Amax, qb_offset,
         nQB if nQB_total is None else nQB_total, _s(stream)))
+
+
+def select_hier(d: PbsaDims, scores, nQB, NB, win_ids, win_frame, n_win, n_frames, F, k, mem_ids,
+                n_mem, blk_len, mask, q_pos0, blk_pos, Tq, idx, cnt, Amax, qb_offset=0,
+                nQB_total=None, stream=None, mem_ld=0):
+    """pbsa_select_hier: frame -> block local selection united with the memory."""
+    _check("pbsa_select_hier", lib().pbsa_select_hier(
+        ctypes.byref(d), _p(scores), nQB, NB, _p(win_ids), _p(win_frame), n_win, n_frames, F, k,
+        _p(mem_ids), n_mem, mem_ld, _p(blk_len), mask, q_pos0, _p(blk_pos), Tq, _p(idx),
+        _p(cnt), Amax, qb_offset, nQB if nQB_total is None else nQB_total, _s(stream)))
 
 
 def route_workspace(d: PbsaDims, P: int, n_cand: int) -> int:

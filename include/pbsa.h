@@ -175,6 +175,42 @@ int pbsa_update_memory(const pbsa_dims* dims, void* kpool, void* vpool, int NB,
                        void* workspace, size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * Backward of a3 for the key and value rows: the recurrent trainable path.
+ * Passage: gist.science/es section 2 "Entrenamiento" (training with the
+ * dynamically updated cache) and the abstract (the memory learns to compress,
+ * keep and refresh persistent blocks): the loss reaches a block's keys and
+ * values also through the slots it was copied or merged into.
+ *
+ * After pbsa_update_memory every slot s is a weighted row-wise sum of
+ * pre-update blocks: unchanged; emptied; a copy of one block (the whole
+ * block); or the merge (bw * base[r < len_base] + sum_m w_m * src_m[r < len_m])
+ * / (bw + sum_m w_m) of its kept block and the losers merged into it (a loser
+ * that was a slot overwritten in the same update is that slot's content before
+ * it).  The selection and merge decisions are constants.  This call applies
+ * the transposed sum:
+ *   on entry dk, dv = the gradient of a loss w.r.t. the pool after the update;
+ *   on return       = the gradient w.r.t. the pool before it: every block keeps
+ *                     its own gradient plus weight * d(slot)[r] (r < rows) for
+ *                     each slot term it appears in; a slot whose content the
+ *                     update replaced or emptied gets only what reaches its
+ *                     pre-update content through such terms; an unchanged slot
+ *                     keeps its gradient.
+ * The rounding of merged rows to the storage type is taken as the identity.
+ *
+ * plan: the first pbsa_update_plan_bytes(dims, P, n_cand) bytes of the
+ * workspace of the pbsa_update_memory call being differentiated, as that call
+ * left them (a rollout keeps a copy per step), 16-byte aligned.  dk, dv: float
+ * [B,H,NB,bs,D], 16-byte aligned.  Candidate ids must lie outside the slot ids
+ * (as in every layout where the window and the slots are apart).
+ * workspace: at least pbsa_update_memory_bwd_workspace(dims, P) bytes,
+ * 256-byte aligned.  Nothing is allocated; asynchronous on `stream`.
+ * ------------------------------------------------------------------------- */
+size_t pbsa_update_plan_bytes(const pbsa_dims* dims, int P, int n_cand);
+size_t pbsa_update_memory_bwd_workspace(const pbsa_dims* dims, int P);
+int pbsa_update_memory_bwd(const pbsa_dims* dims, int NB, int P, int n_cand, const void* plan,
+                           float* dk, float* dv, void* workspace, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
  * a4 + a5: local Top-K selection and the attended-block list.
  * Passage: gist.science/es section 2 "Arquitectura Propuesta", item "Ventana
  * Local" (per-query Top-K of relevant blocks inside the sliding window) and
@@ -210,6 +246,36 @@ int pbsa_select_local(const pbsa_dims* dims, const float* scores, int nQB, int N
                       const int32_t* blk_len, int mask, int q_pos0, const int32_t* blk_pos,
                       int Tq, int32_t* idx, int32_t* cnt, int Amax,
                       int qb_offset, int nQB_total, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * a4 + a5, two-level variant: frame -> block local selection, the alternative
+ * router of the "next" rows.
+ * Passage: Light Forcing (gist.science/it, section 2.2 "Attenzione Sparsa
+ * Gerarchica (HSA)"): keys are mean-pooled per block and per frame; each query
+ * block keeps a few relevant frames by their frame-level keys, then the
+ * critical blocks inside those frames by their block-level keys.
+ *
+ * As pbsa_select_local, except that the local set is chosen in two levels.
+ * A frame is a group of window entries: win_frame[e] in [0, n_frames) is the
+ * frame of entry e (same for every (b,h); n_frames <= 32).  For query block i
+ * the frame's score is the length-weighted mean of scores[b,h,r,j] over its
+ * candidate blocks j (the mean pooled key of the frame's tokens, scored; the
+ * candidates follow the rules of pbsa_select_local), summed in window order;
+ * the F frames of highest score are kept (ties: lower frame), and the local
+ * set is the best min(k, #their candidates) blocks of the kept frames by score
+ * (ties: lower physical id).  The list is its union with the memory ids.  With
+ * F >= n_frames it equals pbsa_select_local's list.
+ * Limits: n_win <= 512, n_mem <= 512, n_mem + min(k, n_win) <= Amax,
+ * NB <= 32768.  win_frame: device int32 [n_win].  Errors as pbsa_select_local
+ * (a win_frame label outside [0, n_frames) sets PBSA_ERR_ARG and the entry is
+ * skipped).
+ * ------------------------------------------------------------------------- */
+int pbsa_select_hier(const pbsa_dims* dims, const float* scores, int nQB, int NB,
+                     const int32_t* win_ids, const int32_t* win_frame, int n_win, int n_frames,
+                     int F, int k, const int32_t* mem_ids, int n_mem, int mem_ld,
+                     const int32_t* blk_len, int mask, int q_pos0, const int32_t* blk_pos,
+                     int Tq, int32_t* idx, int32_t* cnt, int Amax, int qb_offset,
+                     int nQB_total, void* stream);
 
 /* ---------------------------------------------------------------------------
  * a1..a5 in one launch: score -> update memory -> select for one query chunk.

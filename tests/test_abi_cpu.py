@@ -162,3 +162,22 @@ def test_append_rejects_bad_arguments_without_launch():
     # misaligned K rows
     assert lib.pbsa_append_chunk(ctypes.byref(d), ctypes.c_void_p(264), fake, 300, 0, fake, fake,
                                  8, fake, fake, fake, fake, NULL) == -3
+
+
+def test_update_bwd_rejects_bad_arguments_without_launch():
+    lib = _lib.lib()
+    d = _d()
+    fake = ctypes.c_void_p(4096)
+    assert lib.pbsa_update_memory_bwd(ctypes.byref(d), 64, 24, 37, NULL, fake, fake, fake, 1 << 30,
+                                      NULL) == -1
+    assert lib.pbsa_update_memory_bwd(ctypes.byref(d), 8, 24, 37, fake, fake, fake, fake, 1 << 30,
+                                      NULL) == -2            # NB < P
+    assert lib.pbsa_update_memory_bwd(ctypes.byref(d), 64, 24, 37, fake, ctypes.c_void_p(4100),
+                                      fake, fake, 1 << 30, NULL) == -3
+    need = lib.pbsa_update_memory_bwd_workspace(ctypes.byref(d), 24)
+    assert need == 2 * 24 * 2 * 128 * 128 * 4
+    assert lib.pbsa_update_memory_bwd(ctypes.byref(d), 64, 24, 37, fake, fake, fake, fake,
+                                      need - 1, NULL) == -7
+    # the plan is the head of the update workspace
+    assert 0 < lib.pbsa_update_plan_bytes(ctypes.byref(d), 24, 37) <= \
+        lib.pbsa_update_memory_workspace(ctypes.byref(d), 24, 37)
