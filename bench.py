@@ -39,11 +39,11 @@ sys.path.insert(0, ROOT)
 
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
-# DRAM bytes (read + write) of one attn_fwd launch on the decode step, from an
-# ncu capture (profiles/decode_step_kernels_full.md), keyed by a hash of the
-# kernel's sources: a changed kernel reports null until it is captured again.
+# DRAM bytes (read + write) of one attn_fwd launch on the decode step, from a
+# one-launch ncu capture of this workload, keyed by a hash of the kernel's
+# sources: a changed kernel reports null until it is captured again.
 ATTN_TRAFFIC_SOURCES = ["attn_fwd.cu", "tc_sm100.cuh", "common.cuh", "launch.h", "tmap.h"]
-ATTN_TRAFFIC = {"659c99594586ecd3d63a16f49864e45c0e937d163719a42bc00377e713b5cf36": 97268736}
+ATTN_TRAFFIC = {"91216dbb2101212aa8fc26523cbd2ce2c3da31d391134e9960edeac56176a14a": 95695104}
 
 
 def attn_traffic():
@@ -671,6 +671,71 @@ def bench_rollouts(torch):
     return out
 
 
+def bench_select_hier(torch, runner, reps=20):
+    """The two-level (frame -> block) selection against the one-level local
+    selection on the decode step's scores (both per-call, CUDA graphs)."""
+    L, t = runner.L, runner.t
+    out = {}
+    runner.step()
+    torch.cuda.synchronize()
+    out["select_local_ms"] = round(_graph_timed(torch, lambda: L.select(t), reps), 5)
+    for F in (2, 4):
+        out[f"select_hier_F{F}_ms"] = round(
+            _graph_timed(torch, lambda: L.select_hier(t, F, 1560), reps), 5)
+    out["frames"] = "1560-token frames: 3 per chunk, 6 in the 2-chunk window; top-k 16 inside"
+    return out
+
+
+def bench_rollout_backward(torch):
+    """The recurrent trainable path on the 20-second rollout shape (B1 H12 D128,
+    27 chunk steps, merge policy, P48): the forward steps recorded, then the
+    backward of sum_t <O_t, dO_t> back through every step's attention and
+    memory update; per-step time, the attention backward's TF/s over attended
+    blocks (10 len_q len_k D per pair) and the memory update's backward."""
+    import pbsa_inputs as PI
+    from block_sparse_attention_39_b200 import pbsa as K
+    from block_sparse_attention_39_b200.engine import PbsaLayer, PbsaRolloutTrain
+    w = PI.WORKLOADS["rollout20s"]
+    L = PbsaLayer(w)
+    tr = PbsaRolloutTrain(L)
+    dOs = []
+    g = torch.Generator(device="cuda").manual_seed(11)
+    for t in range(w.n_chunks):
+        q, k, v = PI.chunk_tensors_device(w, t)
+        tr.step(t, q, k, v)
+        dOs.append(torch.randn(q.shape, generator=g, device="cuda").bfloat16())
+    torch.cuda.synchronize()
+    tr.backward(dOs)                        # warm-up
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    tr.backward(dOs)
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1)
+    lens = np.array(L.layout.block_lens(), dtype=np.int64)
+    fl = sum(_pair_flops(r["idx"].cpu().numpy(), r["cnt"].cpu().numpy(),
+                         r["blk_len"].cpu().numpy(), lens, w.D, 10) for r in tr.steps)
+    # one memory-update backward on its own
+    rec = [r for r in tr.steps if r["plan"] is not None][-1]
+    dk = torch.zeros(w.B, w.H, L.NB, w.bs, w.D, dtype=torch.float32, device="cuda")
+    dv = torch.zeros_like(dk)
+    upd_ms = _graph_timed(torch, lambda: K.update_memory_bwd(L.d, L.NB, L.P, rec["n_cand"],
+                                                             rec["plan"], dk, dv, tr.upd_ws), 20)
+    merged = int((L.slot_w.cpu().numpy() > 1).sum())
+    out = {"shape": "B1 H12 D128 bf16, 27 steps, P48 merge_mean",
+           "backward_ms_whole_rollout": round(ms, 3),
+           "backward_ms_per_step": round(ms / w.n_chunks, 4),
+           "attn_bwd_tflops_over_attended": round(fl / (ms * 1e-3) / 1e12, 1),
+           "update_memory_bwd_ms": round(upd_ms, 5),
+           "slots_holding_merges_at_end": merged,
+           "note": "includes the per-chunk gradient accumulation (torch adds) and the "
+                   "slot-gradient carry between steps"}
+    del tr, L, dOs
+    torch.cuda.empty_cache()
+    return out
+
+
 def append_traffic(BH, Tc, nb, bs, D):
     """Algorithmic HBM bytes of pbsa_append_chunk (bf16): K and V rows read
     once, their blocks (padding included) written once, the pooled keys and the
@@ -972,6 +1037,8 @@ def main():
         extras["rollouts"] = bench_rollouts(torch)
         extras["hbm_at_scale"] = bench_hbm_at_scale(torch, runner.flush_buf, pk)
         extras["append_chunk"] = bench_append(torch, runner, pk)
+        extras["select_hier"] = bench_select_hier(torch, runner)
+        extras["rollout_backward"] = bench_rollout_backward(torch)
         line["extras"] = extras
     if rank == 0 and not args.no_cpu:
         fl, dt, desc = cpu_oracle_sample(w, runner.chunks)
