@@ -123,6 +123,7 @@ struct RouteParams {
   int t_plan, t_score, t_stash, t_sel, t_apply, t_end;
   int* status;
   int64_t limit_ns;
+  int debug;              // test hook: bit 1 withholds head 0's pool completions
 };
 
 // Per-ticket time stamps for schedule studies, compiled in only with
@@ -198,6 +199,17 @@ __device__ bool wait_count(const RouteParams& r, const unsigned* ctr, unsigned t
 }
 
 // ------------------------------------------------------------------ pooling
+// Counts pool ticket tk done (its mean was written before the caller's last
+// CTA barrier).  Debug bit 1 (pbsa_set_debug) withholds the counts of head 0,
+// so that head's dependent tickets time out: the failure path under test.
+__device__ __forceinline__ void pool_signal(const RouteParams& r, int tk) {
+  const int bh = tk / r.per_pool;
+  if ((r.debug & 2) && bh == 0) return;
+  __threadfence();
+  atomicAdd(r.pool_done + bh, 1u);
+  ROUTE_TRACE(tk, 2);
+}
+
 // The pool tickets, claimed one at a time by thread 0 and streamed through a
 // ring of shared-memory stages (untiled bulk copies completing on mbarriers,
 // the same summation as pool_phase, so the means are bit-identical).  Returns
@@ -264,11 +276,7 @@ __device__ __forceinline__ int route_pool(const RouteParams& r, uint8_t* smem) {
     // thread 0 alone knows how many tickets it has issued
     if (!__syncthreads_or(t == 0 && k < s_ctl[0])) break;
     // the previous item's mean was written before this barrier
-    if (t == 0 && k > 0) {
-      __threadfence();
-      atomicAdd(r.pool_done + prev_tk / r.per_pool, 1u);
-      ROUTE_TRACE(prev_tk, 2);
-    }
+    if (t == 0 && k > 0) pool_signal(r, prev_tk);
     const int s = k % S;
     ok = mbar_wait(smem_u32(&bars[s]), static_cast<uint32_t>((k / S) & 1), abort_flag, a.status,
                    a.limit_ns);
@@ -286,11 +294,7 @@ __device__ __forceinline__ int route_pool(const RouteParams& r, uint8_t* smem) {
     }
   }
   if (ok) {
-    if (t == 0 && k > 0) {
-      __threadfence();
-      atomicAdd(r.pool_done + prev_tk / r.per_pool, 1u);
-      ROUTE_TRACE(prev_tk, 2);
-    }
+    if (t == 0 && k > 0) pool_signal(r, prev_tk);
   } else if (t == 0) {
     atomicExch(r.ctl + 2, 1u);
     // no copy may still be in flight when the stages are reused
@@ -815,7 +819,7 @@ extern "C" int pbsa_route_step(const pbsa_dims* d, const pbsa_route_args* a, voi
   r.t_sel = r.t_stash + (merge ? BH * P_upd : 0);
   r.t_apply = r.t_sel + BH * per_sel;
   r.t_end = r.t_apply + BH * P_upd;
-  r.status = status; r.limit_ns = wait_limit_ns();
+  r.status = status; r.limit_ns = wait_limit_ns(); r.debug = debug_flags();
 
   int launched_rc = PBSA_OK;
   int fallback = 1;

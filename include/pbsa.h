@@ -459,7 +459,10 @@ const char* pbsa_version(void);
  * device wait (nanoseconds; <= 0 restores the default of 2 s) and debug
  * flags: bit 0 makes the next pbsa_attn_fwd launches skip the first V-tile
  * load, so that the tensor-core issuer's wait for it runs out, the kernel
- * sets PBSA_ERR_TIMEOUT and every CTA returns cleanly. */
+ * sets PBSA_ERR_TIMEOUT and every CTA returns cleanly; bit 1 makes the next
+ * pbsa_route_step kernels withhold the completion counts of head 0's pooling,
+ * so that head's dependent work times out, the kernel sets PBSA_ERR_TIMEOUT,
+ * skips the rest, and still leaves its counters zero. */
 void pbsa_set_debug(int flags, int64_t wait_limit_ns);
 
 #ifdef __cplusplus

@@ -146,3 +146,26 @@ def test_route_inside_a_cuda_graph():
     _same_state(La, Lb, "graph")
     assert torch.equal(La.o, Lb.o) and torch.equal(La.lse, Lb.lse)
     _barrier_words_zero(Lb)
+
+
+def test_route_wait_times_out_and_context_survives():
+    # debug bit 1 withholds head 0's pool completions: its plan, score tiles,
+    # lists and slot copies wait on a count that never arrives; with a 20 ms
+    # limit the first waiter aborts the kernel, every CTA skips what is left,
+    # the status word says PBSA_ERR_TIMEOUT and the counters are zero again;
+    # the next call is normal and equals the per-call path
+    w, chunks, t, (La, Lb) = _snapshot_pair("decode")
+    K.get_status()
+    K.set_debug(2, 20_000_000)
+    try:
+        Lb.route(t)
+        assert K.get_status() == -6
+    finally:
+        K.set_debug(0, 0)
+    _barrier_words_zero(Lb)
+    Lb.reset_memory()
+    _per_call(La, t)
+    Lb.route(t)
+    torch.cuda.synchronize()
+    _same_state(La, Lb, "after a timed-out call")
+    _barrier_words_zero(Lb)
