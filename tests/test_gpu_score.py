@@ -2,7 +2,8 @@
 reach: queries of several chunks (a memory score per chunk), chunks that span
 score tiles, one query block per chunk, a single chunk longer than a tile,
 key-block counts that are not tile multiples, empty key blocks, fp32 and bf16,
-D = 64 and 128.
+D = 64 and 128; calls with thousands of score tiles, whose bits must equal
+those of a single head scored alone.
 
 The oracle pools and scores as written (fp64), and its memory score of chunk g
 is the mean of S over the chunk's query blocks.  Tolerances as in the other
@@ -42,6 +43,12 @@ CASES = {
     "one_long_chunk_f32": (1, 1, 128, 128, "f32", 128 * 70, 0, 40, 40),
     # few blocks; only some key blocks re-pooled, the others keep their k_bar
     "small_partial_pool": (1, 2, 64, 128, "bf16", 300, 0, 5, 3),
+    # 259 x 259 blocks per head over 12 heads (2700 score tiles, ragged last
+    # row and column tiles), chunks of 37 blocks
+    "large_d128_bf16": (1, 12, 128, 64, "bf16", 64 * 259 - 5, 64 * 37, 259, 259),
+    # 128 x 330 blocks per head over 25 heads, one chunk spanning every row
+    # tile; some blocks not re-pooled
+    "large_d64_f32": (1, 25, 64, 64, "f32", 64 * 128, 0, 330, 200),
 }
 
 
@@ -90,3 +97,31 @@ def test_score_blocks_shapes_match_oracle(key):
     np.testing.assert_allclose(host(k_bar), kb, rtol=1e-5, atol=1e-6)
     np.testing.assert_allclose(host(scores), S, rtol=1e-4, atol=1e-6)
     np.testing.assert_allclose(host(mem), m, rtol=1e-4, atol=1e-6)
+
+
+def test_large_call_gives_the_single_head_bits():
+    # head (0, 3) of the large case scored alone: every score and memory
+    # score of the twelve-head call must be the same fp32 number (no result
+    # depends on the grid or on other heads)
+    c = _case("large_d128_bf16")
+    scale = 1 / math.sqrt(c["D"])
+    B, H, D, NB, bs, Tq, qc = c["B"], c["H"], c["D"], c["NB"], c["bs"], c["Tq"], c["qc"]
+    nQB = -(-Tq // bs)
+    G = -(-Tq // qc)
+    outs = []
+    for hs in (slice(0, H), slice(3, 4)):
+        h = hs.stop - hs.start
+        d = K.dims(B, h, D, bs, scale, torch.bfloat16, q_chunk=qc)
+        q_bar = torch.zeros(B, h, nQB, D, dtype=torch.float32, device="cuda")
+        k_bar = torch.from_numpy(c["kb0"][:, hs].astype(np.float32)).cuda()
+        scores = torch.zeros(B, h, nQB, NB, dtype=torch.float32, device="cuda")
+        mem = torch.zeros(B, h, G, NB, dtype=torch.float32, device="cuda")
+        K.score_blocks(d, dev_storage(np.ascontiguousarray(c["q"][:, hs]), "bf16"), Tq,
+                       dev_storage(np.ascontiguousarray(c["kp"][:, hs]), "bf16"), NB,
+                       dev_i32(np.ascontiguousarray(c["bl"][:, hs])), dev_i32(c["ids"]),
+                       len(c["ids"]), q_bar, k_bar, scores, mem)
+        torch.cuda.synchronize()
+        outs.append((scores, mem))
+    (s_all, m_all), (s_one, m_one) = outs
+    assert torch.equal(s_all[:, 3:4], s_one)
+    assert torch.equal(m_all[:, 3:4], m_one)
