@@ -61,6 +61,9 @@ int launch_score(const ScoreArgs& a, int BH, cudaStream_t s) {
   if (dev >= 0 && dev < 64 && !attr_set[dev]) {
     cudaFuncSetAttribute(score_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          static_cast<int>(smem));
+    // the whole unified L1 as shared memory, so that six 34 KB tiles fit per SM
+    cudaFuncSetAttribute(score_kernel<D>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                         cudaSharedmemCarveoutMaxShared);
     attr_set[dev] = true;
   }
   dim3 grid(((a.NB + kScoreTile - 1) / kScoreTile) * ((a.nQB + kScoreTile - 1) / kScoreTile), BH);
