@@ -19,7 +19,9 @@ Reported (one JSON line on rank 0):
   --impl reference  times the CPU oracle itself as the reference arm.
 
 Multi-GPU (torchrun): every rank runs its own decode problem (independent
-layers/sequences), no data-path collective; scaling is weak.
+layers/sequences), no data-path collective; scaling is weak.  --shard heads
+instead splits one rollout layer's heads over the ranks and all-gathers the
+output every step (strong scaling).
 """
 from __future__ import annotations
 
@@ -67,6 +69,9 @@ def parse():
                     help="decode: the decode step (default); train: forward + backward of "
                          "the trainable shape on its P32 + top-16 lists; hbm: the score and "
                          "update calls on bandwidth-sized work")
+    ap.add_argument("--shard", default="none", choices=["none", "heads"],
+                    help="heads: one rollout layer split by heads over the ranks, the output "
+                         "all-gathered every step (strong scaling)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-extras", action="store_true",
@@ -910,6 +915,8 @@ def main():
         return run_train(args)
     if args.workload == "hbm":
         return run_hbm(args)
+    if args.shard == "heads":
+        return run_sharded(args)
     import torch
     rank, world, local = init_dist(args.gpus)
     pk, pk_kind = peaks()
@@ -1128,6 +1135,67 @@ def run_hbm(args):
                                        "filling 128 slots of B2 H12; append_chunk of a "
                                        "32 760-token chunk, B2 H12", "parallelism": "replicas"},
                 "calls": res, "peak_kind": pk_kind}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def run_sharded(args):
+    """--shard heads: one layer of the 20-second rollout (B1 H12 D128 bf16, P48
+    merge, window 2 chunks, top-16) split by heads over the ranks, strong
+    scaling.  Every step each rank appends the chunk's K/V for its heads, runs
+    score -> update -> select -> attend on them and all-gathers O over the
+    ranks (NCCL), so every rank ends the step with the whole layer's output.
+    Timed per step with CUDA events on the launching stream (no graphs: the
+    step is the API call a caller makes), max over ranks; the FLOPs are the
+    attended pairs of all heads.  L2 is not flushed: the step's pool and
+    chunk tensors (about 330 MB for 12 heads) exceed the 126 MB L2."""
+    import torch
+    import pbsa_inputs as PI
+    from block_sparse_attention_39_b200.shard import ShardedLayer
+    rank, world, local = init_dist(args.gpus)
+    warm = max(3, args.warmup, PI.WORKLOADS["rollout20s"].W + 2)
+    steps = max(1, args.steps)
+    w = PI.variant(PI.WORKLOADS["rollout20s"], n_chunks=warm + steps)
+    S = ShardedLayer(w, world, rank)
+    L = S.layer
+    q_lens = np.array(L.layout.block_lens(), dtype=np.int64)
+    ms, flops = [], 0
+    for t in range(warm + steps):
+        q, k, v = PI.chunk_tensors_device(w, t)
+        torch.cuda.synchronize()
+        barrier(world)
+        e0, e1 = (torch.cuda.Event(enable_timing=True) for _ in range(2))
+        e0.record()
+        S.step(t, q, k, v)
+        e1.record()
+        torch.cuda.synchronize()
+        if t >= warm:
+            ms.append(e0.elapsed_time(e1))
+            flops += _pair_flops(L.idx.cpu().numpy(), L.cnt.cpu().numpy(),
+                                 L.blk_len.cpu().numpy(), q_lens, w.D, 4)
+    ms_step = max_over_ranks(float(np.mean(ms)), world)
+    if world > 1:
+        import torch.distributed as dist
+        ft = torch.tensor([float(flops)], dtype=torch.float64, device="cuda")
+        dist.all_reduce(ft)
+        flops = ft.item()
+    value = flops / steps / (ms_step * 1e-3) / 1e12
+    if rank == 0:
+        line = {"metric": "PBSA fwd effective TFLOP/s (attended blocks) & per-chunk latency",
+                "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world, "steps": steps,
+                "warmup": warm, "ms_per_step": round(ms_step, 5), "higher_is_better": True,
+                "scaling": "strong", "vs_baseline": None, "dtype": "bf16",
+                "data": "synthetic (seeded N(0,1) Q/K/V drawn on the device, salient blocks)",
+                "config": {"workload": f"one layer of the 20-second rollout, B{w.B} H{w.H} "
+                                       f"D{w.D} bf16, P{w.P} merge, W{w.W} chunks, k{w.k}, "
+                                       f"steps {warm}..{warm + steps - 1}",
+                           "global_batch": w.B, "seq_len": w.chunk_tokens,
+                           "l2": "not flushed: the step's data exceed the 126 MB L2",
+                           "parallelism": f"heads{world}"},
+                "timed": "one step per pair of CUDA events: append, score, update, select, "
+                         "attend and the all-gather of O"}
         print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist
